@@ -1,0 +1,377 @@
+#!/usr/bin/env python
+"""Throughput of the ViT encoder forward on B200: images/s and the roofline of its top kernel.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
+
+One step = one vit_forward over one batch of the workload (default: DINOv3-style ViT-L/16 at
+1024 x 1024, batch 8 per GPU, seeded synthetic weights and images).  Ranks are independent
+replicas (weak scaling: images of different ranks never interact); torch.distributed over
+NCCL is used only for the barrier and the max-over-ranks time.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle instead (rank 0 only), each step a bounded
+sample of the same workload, scaled to images/s.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as S  # noqa: E402
+
+METRIC = "images/s ViT-S/16@336 & ViT-L/16@1024 bf16, 1 B200; % of bf16 tensor peak"
+WORKLOAD_TEXT = {
+    "vitl16_1024_b8": "ViT-L/16@1024 DINOv3-style (CLS + 4 registers + 4096 patches = 4101 tokens), batch 8",
+    "vitl16_1024_b1": "ViT-L/16@1024 DINOv3-style (4101 tokens), batch 1",
+    "vits16_336_b1": "ViT-S/16@336 DINOv3-style (446 tokens), batch 1",
+    "vits16_336_b64_outlier": "ViT-S/16@336 DINOv3-style with attention-sink outlier (446 tokens), batch 64",
+    "vits14_518_b8_taps": "ViT-S/14@518 DINOv2-style (1370 tokens) with taps 3/6/9/12, batch 8",
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# Algorithmic FLOPs (2 per multiply-add) of each kernel kind for one launch over B images.
+def kernel_flops(spec, B):
+    T, P, D, F, p = spec.tokens, spec.n_patches, spec.dim, spec.mlp, spec.patch
+    M = B * T
+    return {
+        "patch_gemm": 2.0 * B * P * D * 3 * p * p,
+        "qkv_gemm": 2.0 * M * 3 * D * D,
+        "attention": 4.0 * B * T * T * D,
+        "proj_gemm": 2.0 * M * D * D,
+        "fc1_gemm": 2.0 * M * F * D,
+        "fc2_gemm": 2.0 * M * D * F,
+    }
+
+
+def total_flops(spec, B):
+    f = kernel_flops(spec, B)
+    return f["patch_gemm"] + spec.depth * (f["qkv_gemm"] + f["attention"] + f["proj_gemm"] + f["fc1_gemm"] + f["fc2_gemm"])
+
+
+# Algorithmic bytes of the memory-bound kinds for one launch over B images.
+def kernel_bytes(spec, B):
+    T, P, D = spec.tokens, spec.n_patches, spec.dim
+    return {
+        "im2col": B * 3 * spec.img_h * spec.img_w * 4 + B * P * (((3 * spec.patch ** 2 + 63) // 64) * 64) * 2,
+        "final_ln": B * (1 + P) * D * 4 + B * P * D * 2 + B * D * 4,
+        "prefix": B * (1 + spec.registers) * D * 6,
+        "tap": B * P * D * 8,
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while the timed region runs."""
+
+    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown," \
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+             "clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_sample(spec, weights, images, blocks):
+    """Time the fp64 oracle on one image through `blocks` encoder blocks; returns seconds."""
+    import oracle as O
+    t0 = time.perf_counter()
+    O.forward(images[:1], weights, spec, n_blocks=blocks)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    """The oracle as it stands, on a bounded sample of the workload: one image through as many
+    encoder blocks as fit in about `budget_s` seconds, scaled to images/s for the full depth."""
+    import oracle as O
+    spec = wl.spec
+    weights = O.to_f64_weights(S.make_weights(spec, wl.weight_seed, wl.outlier))
+    images = S.make_images(spec, 1, wl.image_seed)
+    t1 = oracle_sample(spec, weights, images, 1)
+    n = max(1, min(spec.depth, int(budget_s / max(t1, 1e-3))))
+    tn = oracle_sample(spec, weights, images, n) if n > 1 else t1
+    per_image = tn * spec.depth / n
+    return {"value": 1.0 / per_image, "unit": "images/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"1 image of {wl.name} through {n} of {spec.depth} blocks in {tn:.2f} s (fp64 numpy), "
+                      f"scaled by depth"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle as O
+    wl = S.WORKLOADS[args.workload]
+    spec = wl.spec
+    weights = O.to_f64_weights(S.make_weights(spec, wl.weight_seed, wl.outlier))
+    images = S.make_images(spec, 1, wl.image_seed)
+    blocks = 1
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = oracle_sample(spec, weights, images, blocks)
+        if i >= args.warmup:
+            times.append(t)
+    per_image = statistics.mean(times) * spec.depth / blocks
+    value = 1.0 / per_image
+    cores = blas_threads()
+    sample = f"each step: 1 image of {wl.name} through {blocks} of {spec.depth} blocks (fp64 numpy), scaled by depth"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "images/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT.get(wl.name, wl.name), "batch_per_gpu": wl.batch,
+                       "parallelism": "oracle on host cores"},
+            "cpu_baseline": {"value": value, "unit": "images/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "images/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def secondary_rate(V, name, steps=20, warmup=5):
+    """images/s of another workload on this GPU (device-timed, no host copies)."""
+    spec, w, im = S.make_workload(name)
+    enc = V.VitEncoder(spec, w, max_batch=im.shape[0])
+    x = im.cuda()
+    outs = enc.alloc_outputs(x.shape[0], desc=True, patch=True)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        enc.forward_into(x, outs)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        enc.forward_into(x, outs)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    enc.poll()
+    ms = e0.elapsed_time(e1) / steps
+    enc.close()
+    return {"workload": WORKLOAD_TEXT.get(name, name), "images_per_s": x.shape[0] / (ms / 1000.0),
+            "ms_per_step": ms, "tflops": total_flops(spec, x.shape[0]) / (ms / 1000.0) / 1e12}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="vitl16_1024_b8", choices=sorted(WORKLOAD_TEXT))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import vision_transformer_encoder_fwd_b200 as V
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    wl = S.WORKLOADS[args.workload]
+    spec = wl.spec
+    B = wl.batch
+    weights = S.make_weights(spec, wl.weight_seed, wl.outlier)
+    enc = V.VitEncoder(spec, weights, max_batch=B)
+    # two input buffers alternate between steps (2 x 100 MB for ViT-L b8: more than the 126 MB L2)
+    imgs = [S.make_images(spec, B, wl.image_seed + 1000 * rank + k).cuda() for k in range(2)]
+    outs = enc.alloc_outputs(B, desc=True, patch=True, patch_fp32=False)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        enc.forward_into(imgs[i % 2], outs)
+    torch.cuda.synchronize()
+    enc.poll()
+
+    # ---- timed region (device time, CUDA events on the launching stream; per-launch events inside)
+    launches_per_step = enc.last_launch_count()
+    enc.profile_begin(launches_per_step * args.steps + 16)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        enc.forward_into(imgs[i % 2], outs)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    prof = enc.profile_end()
+    enc.poll()
+    ms_total = e0.elapsed_time(e1)
+    t = torch.tensor([ms_total], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    value = world * B * args.steps / (ms_total / 1000.0)
+
+    # ---- end to end through vit_forward_host: pinned host images in, descriptor + patch tokens out
+    host_imgs = [im.cpu().pin_memory() for im in imgs]
+    desc_h = torch.empty(B, spec.dim, dtype=torch.float32).pin_memory()
+    patch_h = torch.empty(B, spec.n_patches, spec.dim, dtype=torch.bfloat16).pin_memory()
+    hws = torch.empty(enc.host_workspace_size(B), dtype=torch.uint8, device="cuda")
+    for i in range(args.warmup):
+        enc.forward_host(host_imgs[i % 2], desc_h, patch_h, ws=hws)
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(args.steps):
+        enc.forward_host(host_imgs[i % 2], desc_h, patch_h, ws=hws)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    enc.poll()
+    t2 = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+    e2e_value = world * B * args.steps / (float(t2.item()) / 1000.0)
+    h2d = host_imgs[0].numel() * 4
+    d2h = desc_h.numel() * 4 + patch_h.numel() * 2
+
+    peaks = load_peaks()
+    line = None
+    if rank == 0:
+        flops = kernel_flops(spec, B)
+        nbytes = kernel_bytes(spec, B)
+        kernels = {}
+        for k, (ms, n) in prof.items():
+            entry = {"launches": n, "total_ms": ms, "avg_ms": ms / n, "share": ms / max(1e-9, sum(v[0] for v in prof.values()))}
+            if k in flops:
+                entry["tflops"] = flops[k] / (ms / n / 1000.0) / 1e12
+            if k in nbytes:
+                entry["gbs"] = nbytes[k] / (ms / n / 1000.0) / 1e9
+            kernels[k] = entry
+        top = max(prof, key=lambda k: prof[k][0])
+        avg_s = prof[top][0] / prof[top][1] / 1000.0
+        if top in flops:
+            ach = flops[top] / avg_s / 1e12
+            peak = peaks["bf16_tflops_sustained"]
+            roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                    "traffic": None, "kernel": top, "flops_per_launch": flops[top],
+                    "peak_kind": f"bf16 dense, sustained ({peaks['source']})"}
+        else:
+            ach = nbytes.get(top, 0) / avg_s / 1e9
+            peak = peaks["hbm_gbs"]
+            roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                    "traffic": None, "kernel": top, "peak_kind": f"HBM copy ({peaks['source']})"}
+        step_flops = total_flops(spec, B)
+        line = {
+            "metric": METRIC, "value": value, "unit": "images/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT[wl.name], "batch_per_gpu": B, "global_batch": B * world,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "two input buffers alternate (2 x %.0f MB); weights %.0f MB and activations per step "
+                             "exceed the 126 MB L2" % (imgs[0].numel() * 4 / 1e6, sum(
+                                 p.numel() * 2 for p in enc.w.values()) / 1e6 + sum(
+                                 p.numel() * 2 for b in enc.wb for p in b.values()) / 1e6),
+                       "timing": "CUDA events on the launching stream; per-launch events recorded inside the "
+                                 "timed region for the kernel breakdown"},
+            "tflops_per_gpu": step_flops / (ms_total / args.steps / 1000.0) / 1e12,
+            "frac_of_bf16_peak": {"measured_burst": step_flops / (ms_total / args.steps / 1000.0) / 1e12 /
+                                  peaks["bf16_tflops"], "spec_dense_2250": step_flops / (
+                                      ms_total / args.steps / 1000.0) / 1e12 / 2250.0},
+            "roofline": roof,
+            "kernels": kernels,
+            "e2e": {"value": e2e_value, "unit": "images/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+        }
+    enc.close()
+    if rank == 0:
+        if not args.no_secondary:
+            line["secondary"] = [secondary_rate(V, "vits16_336_b64_outlier"), secondary_rate(V, "vits16_336_b1")]
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

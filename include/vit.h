@@ -1,0 +1,194 @@
+/*
+ * vit.h -- C ABI of libvit_b200: the DINOv2/DINOv3 ViT encoder forward on one B200 (sm_100a).
+ *
+ * The interface follows the kornia/dinov3 model card ("Usage"): build a model from weights,
+ * let the caller own the result buffers, enqueue the forward on a stream without
+ * synchronising, and read an L2-normalised descriptor.  Errors come back as status codes,
+ * never as process aborts; nothing here traps on the device.
+ *
+ * Pages cited (title, section / panel):
+ *   [card]    "kornia/dinov3" model card: "Model I/O", "Build BF16, not FP16", "Usage".
+ *   [diagram] "DINOv2 n semantic" architecture diagram: "DINOv2-S encoder", "Encoder block",
+ *             "Encoder self-attention".
+ *   [dinotxt] "DINOv3零样本分割实测：dino.txt补丁级匹配与双推理模式": patch/text alignment and
+ *             the whole / slide inference modes.
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" are CUDA device memory of the current device; "host" are host
+ *     memory (pinned memory makes the copies asynchronous).  All device pointers must be
+ *     16-byte aligned.  The caller owns all memory passed in; the library never frees it.
+ *   - bf16 means IEEE bfloat16 (2 bytes); matrices are row-major, nn.Linear weights [out, in].
+ *   - Functions taking a cudaStream_t enqueue work on that stream and return without
+ *     synchronising (except where stated).  Host validation happens before any launch; on a
+ *     validation failure nothing is enqueued.
+ *   - Device-side failures (a pipeline wait that ran out of time) set the model's status
+ *     word; vit_poll() reads it.  No kernel traps.
+ */
+#ifndef VIT_B200_H
+#define VIT_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *vit_stream_t; /* == cudaStream_t; NULL = legacy default stream */
+
+typedef enum vit_status {
+  VIT_OK = 0,
+  VIT_E_INVALID_ARG = 1,    /* null / misaligned pointer, bad value */
+  VIT_E_SHAPE = 2,          /* sizes inconsistent with the model or with each other */
+  VIT_E_UNSUPPORTED = 3,    /* a configuration this build does not implement */
+  VIT_E_WORKSPACE = 4,      /* workspace smaller than vit_*_workspace_size reports */
+  VIT_E_CUDA = 5,           /* a CUDA runtime / driver call failed */
+  VIT_E_DEVICE_TIMEOUT = 6, /* a device pipeline wait gave up (read via vit_poll) */
+  VIT_E_NONFINITE = 7       /* reserved: non-finite value detected */
+} vit_status;
+
+/* Encoder architecture.  [diagram] "DINOv2-S encoder" / "Encoder block"; [card] "Model I/O".
+ * Constraints checked by vit_create: head width dim/heads == 64; dim and mlp_dim multiples of
+ * 128; img_h, img_w multiples of patch; 1 <= patch <= 32; 0 <= n_registers <= 16;
+ * 1 <= depth <= 64; max_batch >= 1; ln_eps > 0; at most 4 taps, all <= depth. */
+typedef struct vit_config {
+  int32_t patch;       /* p: patch side (16 DINOv3, 14 DINOv2) */
+  int32_t img_h;       /* native input height in pixels (multiple of p) */
+  int32_t img_w;       /* native input width in pixels (multiple of p) */
+  int32_t dim;         /* D: token width */
+  int32_t depth;       /* L: number of encoder blocks */
+  int32_t heads;       /* D / 64 */
+  int32_t mlp_dim;     /* F: MLP hidden width (4 D) */
+  int32_t n_registers; /* R: register tokens between CLS and the patches (4 DINOv3, 0 DINOv2) */
+  int32_t pos_on_cls;  /* 1: position embedding has 1 + P rows, row 0 added to CLS (DINOv2);
+                          0: P rows, patches only (DINOv3) */
+  int32_t max_batch;   /* largest batch vit_forward will be called with */
+  float ln_eps;        /* LayerNorm eps (1e-6) */
+  uint32_t tap_mask;   /* bit (l-1) set: tap after block l ([diagram] taps 3/6/9/12) */
+} vit_config;
+
+/* One encoder block's weights: device pointers to bf16 ([diagram] "Encoder block",
+ * "Encoder self-attention").  The Q, K and V Linears are stacked: qkv_w [3D, D] with rows
+ * q (0..D-1) | k (D..2D-1) | v (2D..3D-1); head h owns rows 64h..64h+63 of each part. */
+typedef struct vit_block_weights {
+  const void *ln1_w, *ln1_b;   /* [D] */
+  const void *qkv_w, *qkv_b;   /* [3D, D], [3D] */
+  const void *proj_w, *proj_b; /* [D, D], [D] */
+  const void *ls1;             /* [D] layer scale of the attention branch */
+  const void *ln2_w, *ln2_b;   /* [D] */
+  const void *fc1_w, *fc1_b;   /* [F, D], [F] */
+  const void *fc2_w, *fc2_b;   /* [D, F], [D] */
+  const void *ls2;             /* [D] layer scale of the MLP branch */
+} vit_block_weights;
+
+/* Whole-model weights: device pointers to bf16, except `blocks`, a HOST array of `depth`
+ * entries.  Borrowed: the device memory must stay valid and unchanged for the model's life.
+ * The model also keeps derived copies it allocates itself (see vit_create). */
+typedef struct vit_weights {
+  const void *patch_w;  /* [D, 3, p, p] Conv2d weight */
+  const void *patch_b;  /* [D] */
+  const void *cls;      /* [D] learned CLS token */
+  const void *reg;      /* [R, D] register tokens; may be NULL when R == 0 */
+  const void *pos;      /* [pos_on_cls + gh*gw, D] learned additive position embedding */
+  const void *norm_w, *norm_b; /* [D] final LayerNorm (also applied to the taps) */
+  const vit_block_weights *blocks; /* host array [depth] */
+} vit_weights;
+
+/* Outputs of vit_forward; every pointer is optional (NULL = not wanted).  Device memory. */
+typedef struct vit_outputs {
+  float *desc;          /* [B, D] fp32: final-LN CLS token / max(||.||_2, 1e-12) ([card]) */
+  void *patch_tokens;   /* [B, gh*gw, D] final-LN patch tokens (CLS and registers dropped),
+                           fp32 if patch_fp32 else bf16 */
+  int32_t patch_fp32;
+  float *taps[4];       /* [B, D, gh, gw] fp32 each: final LayerNorm of the tokens after the
+                           tapped blocks in ascending order, CLS and registers removed,
+                           channels first ([diagram] "Taps apply LayerNorm, remove CLS, reshape") */
+  float *hidden;        /* [depth, B, T, D] fp32 residual stream after every block
+                           (T = 1 + R + gh*gw); a diagnostic for parity checks */
+} vit_outputs;
+
+typedef struct vit_model vit_model;
+
+/* Validate the configuration, borrow the weights and prepare the derived weights the kernels
+ * consume: the LayerNorm gammas folded into the QKV and FC1 matrices (bf16), the betas folded
+ * into their biases (fp32), column sums of the folded matrices, the patch matrix padded to a
+ * multiple of 64 columns, and fp32 copies of the vectors.  Runs on the current device and
+ * synchronises it once.  On success *out receives the model. */
+vit_status vit_create(const vit_config *cfg, const vit_weights *w, vit_model **out);
+
+/* Bytes of device workspace vit_forward needs for `batch` images (batch <= max_batch). */
+vit_status vit_workspace_size(const vit_model *m, int32_t batch, size_t *bytes);
+
+/* The encoder forward ([diagram] "DINOv2-S encoder" with its blocks; [card] "Model I/O"):
+ *   images  device fp32 [B, 3, img_h, img_w], ImageNet-normalised (the caller normalises);
+ *           rounded to bf16 by the patch-embedding kernel.
+ *   B       1 <= B <= max_batch.
+ *   ws      device workspace of at least vit_workspace_size(m, B) bytes, 256-byte aligned;
+ *           it must not be used concurrently by another call.
+ * Enqueues on `stream`; returns without synchronising. */
+vit_status vit_forward(vit_model *m, const float *images, int32_t B, const vit_outputs *out,
+                       void *ws, size_t ws_bytes, vit_stream_t stream);
+
+/* The same forward from host memory: copies `images_host` [B, 3, img_h, img_w] fp32 into the
+ * workspace, runs vit_forward, and copies the descriptor [B, D] fp32 to `desc_host` and (if
+ * non-NULL) the bf16 patch tokens [B, gh*gw, D] to `patch_tokens_host`.  Needs
+ * vit_host_workspace_size bytes.  Enqueues on `stream`; the host buffers must stay valid until
+ * the stream has been synchronised (pinned host memory makes the copies asynchronous). */
+vit_status vit_host_workspace_size(const vit_model *m, int32_t batch, size_t *bytes);
+vit_status vit_forward_host(vit_model *m, const float *images_host, int32_t B, float *desc_host,
+                            void *patch_tokens_host, void *ws, size_t ws_bytes, vit_stream_t stream);
+
+/* Zero-shot dense scoring ([dinotxt] patch/text alignment; whole and slide modes). */
+enum { VIT_SEG_WHOLE = 0, VIT_SEG_SLIDE = 1 };
+
+/* Workspace for vit_seg_zero_shot with these arguments. */
+vit_status vit_seg_workspace_size(const vit_model *m, int32_t H, int32_t W, int32_t C, int32_t mode,
+                                  int32_t side, int32_t stride, size_t *bytes);
+
+/* image  device fp32 [3, H, W], ImageNet-normalised.
+ * text   device fp32 [C, D] class embeddings (unit rows; used as given).
+ * WHOLE: H, W must equal the model's img_h, img_w (the position embedding is not resized);
+ *        the encoder runs once; scores = bilinear (align_corners=False) upsample of the cosine
+ *        map cos[c, i] = text[c] . t_i / max(||t_i||, 1e-12) over the final-LN patch tokens t.
+ * SLIDE: side must equal img_h == img_w; windows of side x side at `stride`, per axis
+ *        ceil((size - side) / stride) + 1 origins with the last clamped to size - side; every
+ *        window runs the encoder (all windows in one batch, so max_batch must cover them);
+ *        per window the cosine map is upsampled to side x side, softmaxed over classes and
+ *        accumulated; the sum is divided by the per-pixel window count.
+ * probs  device fp32 [C, H, W] (scores in WHOLE mode, averaged probabilities in SLIDE) or NULL.
+ * labels device int32 [H, W] argmax over classes (lowest index on ties) or NULL.
+ * Enqueues on `stream`. */
+vit_status vit_seg_zero_shot(vit_model *m, const float *image, int32_t H, int32_t W, const float *text,
+                             int32_t C, int32_t mode, int32_t side, int32_t stride, float *probs,
+                             int32_t *labels, void *ws, size_t ws_bytes, vit_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the model's device status word.  Returns VIT_OK,
+ * VIT_E_DEVICE_TIMEOUT if a kernel gave up on a pipeline wait since the last poll, or
+ * VIT_E_CUDA if the stream reports an error. */
+vit_status vit_poll(vit_model *m, vit_stream_t stream);
+
+/* Number of kernel launches the last vit_forward / vit_seg_zero_shot call made. */
+int32_t vit_last_launch_count(const vit_model *m);
+
+/* Per-launch timing on the caller's stream.  After vit_profile_begin(m, capacity) every kernel
+ * launch of vit_forward / vit_seg_zero_shot (up to `capacity` launches in total) is bracketed by
+ * two CUDA events recorded on the launch stream.  vit_profile_end synchronises those events,
+ * adds up the elapsed times per kernel kind into total_ms[VIT_K_COUNT] (milliseconds) and
+ * launches[VIT_K_COUNT], and switches profiling off.  Either output pointer may be NULL. */
+enum {
+  VIT_K_IM2COL = 0, VIT_K_PATCH_GEMM, VIT_K_PREFIX, VIT_K_QKV_GEMM, VIT_K_ATTENTION, VIT_K_PROJ_GEMM,
+  VIT_K_FC1_GEMM, VIT_K_FC2_GEMM, VIT_K_TAP, VIT_K_FINAL_LN, VIT_K_SEG_NORM, VIT_K_SEG_COS, VIT_K_SEG_MAP,
+  VIT_K_COUNT
+};
+vit_status vit_profile_begin(vit_model *m, int32_t capacity);
+vit_status vit_profile_end(vit_model *m, float *total_ms, int32_t *launches);
+
+void vit_destroy(vit_model *m);
+const char *vit_status_str(vit_status s);
+/* Text of the last host-side error of this thread (validation message or CUDA error). */
+const char *vit_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VIT_B200_H */

@@ -1,0 +1,36 @@
+/*
+ * vit_stages.h -- stage-level entry points of libvit_b200, exposed so that each hot kernel can
+ * be checked on its own against the fp64 oracle.  They run the same kernels vit_forward runs.
+ *
+ * Conventions as in vit.h: device pointers, 16-byte aligned, caller-owned; work is enqueued on
+ * `stream` without synchronising; `status` is a caller-allocated device int32 (zero-initialised)
+ * that a kernel sets to a non-zero code if one of its pipeline waits gives up, and that every
+ * kernel checks on entry (a non-zero status makes later kernels return without work).
+ */
+#ifndef VIT_B200_STAGES_H
+#define VIT_B200_STAGES_H
+
+#include "vit.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* out[M, N] = act(A[M, K] . W[N, K]^T + bias[N]) on the tcgen05 GEMM ("DINOv2 n semantic"
+ * diagram, "Encoder block": the Linear layers; act = exact-erf GELU when gelu != 0).
+ *   A, W: bf16, row-major, K contiguous;  bias: fp32 [N];  out: bf16 [M, N].
+ *   Requires M >= 1, N a multiple of 128, K a multiple of 64.  VIT_E_SHAPE otherwise. */
+vit_status vit_stage_linear(const void *A, const void *W, const float *bias, int32_t M, int32_t N, int32_t K,
+                            int32_t gelu, void *out, int32_t *status, vit_stream_t stream);
+
+/* Multi-head self-attention core ("DINOv2 n semantic" diagram, "Encoder self-attention"):
+ * for each image b and head h, out[b, :, 64h:64h+64] = softmax_keys(Q_h K_h^T / 8) V_h with
+ * Q_h, K_h, V_h the 64-column slices h of the q, k and v parts of qkv[b] = [q | k | v].
+ *   qkv: bf16 [B, T, 3 * 64 * heads];  out: bf16 [B, T, 64 * heads].  T >= 1, heads >= 1. */
+vit_status vit_stage_attention(const void *qkv, int32_t B, int32_t T, int32_t heads, void *out, int32_t *status,
+                               vit_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VIT_B200_STAGES_H */

@@ -272,3 +272,9 @@ def as_numpy_f64(t) -> np.ndarray:
     if isinstance(t, np.ndarray):
         return t.astype(np.float64)
     return t.detach().to(torch.float64).cpu().numpy()
+
+
+def make_matrix(shape, seed: int, std: float = 1.0, dtype=torch.bfloat16) -> torch.Tensor:
+    """N(0, std^2) draws of the given shape, rounded to ``dtype`` (stage-level test inputs)."""
+    g = torch.Generator().manual_seed(int(seed))
+    return (torch.randn(*shape, generator=g, dtype=torch.float32) * std).to(dtype)

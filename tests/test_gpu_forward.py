@@ -1,0 +1,102 @@
+"""End-to-end parity of vit_forward against the fp64 oracle, per configuration.
+
+Small shapes are compared on every image; the full-size workloads run in the launch
+configuration the bench times (whole batch on the GPU) and are compared on sampled images,
+which the oracle computes one by one."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synthetic as S
+from parity import assert_forward_parity, gpu, need_cuda, run_gpu
+
+pytestmark = gpu
+
+
+@pytest.mark.parametrize("name,batch", [("tiny_s16", 2), ("tiny_s14", 3), ("small_s16", 2)])
+def test_small_configs_all_images(name, batch):
+    need_cuda()
+    spec = S.PRESETS[name]
+    w = S.make_weights(spec, 31)
+    im = S.make_images(spec, batch, 32)
+    g = run_gpu(spec, w, im)
+    ref = O.forward(im, w, spec, record_hidden=True)
+    assert_forward_parity(g, ref, spec, list(range(batch)))
+
+
+def test_vits16_336_b1():
+    need_cuda()
+    spec, w, im = S.make_workload("vits16_336_b1")
+    g = run_gpu(spec, w, im)
+    ref = O.forward(im, w, spec, record_hidden=True)
+    assert_forward_parity(g, ref, spec, [0])
+
+
+def test_vits16_336_b64_attention_sink():
+    """kornia/dinov3 card, "Build BF16, not FP16": block-1 logits of ~2.2e6, no NaN anywhere."""
+    need_cuda()
+    spec, w, im = S.make_workload("vits16_336_b64_outlier")
+    g = run_gpu(spec, w, im)
+    assert np.isfinite(g["hidden"]).all() and np.isfinite(g["desc"]).all()
+    idx = [0, 37, 63]
+    ref = O.forward(im, w, spec, record_hidden=True, image_indices=idx)
+    assert_forward_parity(g, ref, spec, idx)
+
+
+def test_vits14_518_b8_taps():
+    need_cuda()
+    spec, w, im = S.make_workload("vits14_518_b8_taps")
+    g = run_gpu(spec, w, im)
+    for t in g["taps"]:
+        assert t.shape == (8, 384, 37, 37)
+    idx = [0, 7]
+    ref = O.forward(im, w, spec, record_hidden=True, image_indices=idx)
+    assert_forward_parity(g, ref, spec, idx)
+
+
+@pytest.mark.slow
+def test_vitl16_1024_b8():
+    need_cuda()
+    spec, w, im = S.make_workload("vitl16_1024_b8")
+    g = run_gpu(spec, w, im, hidden=True)
+    assert np.isfinite(g["hidden"]).all()
+    idx = [5]
+    ref = O.forward(im, w, spec, record_hidden=True, image_indices=idx)
+    assert_forward_parity(g, ref, spec, idx)
+
+
+def test_forward_host_matches_device_path():
+    need_cuda()
+    import vision_transformer_encoder_fwd_b200 as V
+    spec = S.PRESETS["small_s16"]
+    w = S.make_weights(spec, 41)
+    im = S.make_images(spec, 3, 42)
+    enc = V.VitEncoder(spec, w, max_batch=3)
+    dev = enc.forward(im.cuda(), desc=True, patch=True)
+    ih = im.pin_memory()
+    dh = torch.empty(3, spec.dim, dtype=torch.float32).pin_memory()
+    ph = torch.empty(3, spec.n_patches, spec.dim, dtype=torch.bfloat16).pin_memory()
+    enc.forward_host(ih, dh, ph)
+    torch.cuda.synchronize()
+    enc.poll()
+    assert torch.equal(dh, dev["desc"].cpu())
+    assert torch.equal(ph, dev["patch_tokens"].cpu())
+    enc.close()
+
+
+def test_repeated_calls_are_deterministic_and_launch_count():
+    need_cuda()
+    import vision_transformer_encoder_fwd_b200 as V
+    spec = S.PRESETS["tiny_s14"]
+    w = S.make_weights(spec, 51)
+    im = S.make_images(spec, 2, 52).cuda()
+    enc = V.VitEncoder(spec, w, max_batch=2)
+    a = enc.forward(im, desc=True, patch=True, taps=True)
+    b = enc.forward(im, desc=True, patch=True, taps=True)
+    torch.cuda.synchronize()
+    enc.poll()
+    assert torch.equal(a["desc"], b["desc"]) and torch.equal(a["patch_tokens"], b["patch_tokens"])
+    # im2col, patch GEMM, prefix rows, 5 per block, one per tap, final LayerNorm
+    assert enc.last_launch_count() == 3 + 5 * spec.depth + len(spec.taps) + 1
+    enc.close()

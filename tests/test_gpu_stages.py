@@ -1,0 +1,102 @@
+"""Stage-level parity of the hot kernels through the C ABI (vit_stage_linear,
+vit_stage_attention) against the fp64 oracle's building blocks on the same bf16 inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synthetic as S
+from parity import gpu, need_cuda
+
+pytestmark = gpu
+
+
+def _ref_linear(A, W, b, gelu):
+    r = A.double().numpy() @ W.double().numpy().T + b.double().numpy()
+    return O.gelu(r) if gelu else r
+
+
+@pytest.mark.parametrize("M,N,K,gelu", [
+    (1, 128, 64, False),        # one row, one tile
+    (129, 384, 384, False),     # ragged second M tile
+    (446, 1152, 384, False),    # ViT-S/16 QKV shape
+    (446, 1536, 384, True),     # ViT-S/16 FC1 with GELU
+    (1000, 1024, 4096, False),  # long K (FC2-like), ragged M
+    (5000, 4096, 1024, True),   # 256-column tiles (enough tiles to fill the SMs)
+])
+def test_linear_matches_oracle(M, N, K, gelu):
+    need_cuda()
+    import vision_transformer_encoder_fwd_b200 as V
+    A = S.make_matrix((M, K), 1 + M, 1.0)
+    W = S.make_matrix((N, K), 2 + N, 1.0 / math.sqrt(K))
+    b = S.make_matrix((N,), 3, 0.5, torch.float32)
+    out, st = V.stage_linear(A.cuda(), W.cuda(), b.cuda(), gelu=gelu)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    g = out.double().cpu().numpy()
+    r = _ref_linear(A, W, b, gelu)
+    assert np.isfinite(g).all()
+    err = np.abs(g - r).max()
+    assert err <= 6e-3 * np.abs(r).max() + 1e-3, err
+
+
+def _ref_attention(qkv, heads):
+    B, T, _ = qkv.shape
+    D = heads * 64
+    x = qkv.double().numpy()
+    out = np.empty((B, T, D))
+    for b in range(B):
+        for h in range(heads):
+            q = x[b, :, h * 64:(h + 1) * 64]
+            k = x[b, :, D + h * 64:D + (h + 1) * 64]
+            v = x[b, :, 2 * D + h * 64:2 * D + (h + 1) * 64]
+            out[b, :, h * 64:(h + 1) * 64] = O.attention_probs(q, k) @ v
+    return out
+
+
+@pytest.mark.parametrize("B,T,heads,qk_scale", [
+    (1, 1, 1, 1.0),       # a single key: output = v
+    (2, 65, 2, 1.0),      # one ragged KV tile
+    (1, 129, 1, 3.0),     # two KV tiles, the second with one key; sharper softmax
+    (1, 446, 6, 1.0),     # ViT-S/16@336 tokens
+    (2, 1370, 6, 2.0),    # ViT-S/14@518 tokens
+    (1, 4101, 2, 1.0),    # ViT-L/16@1024 tokens (two heads)
+])
+def test_attention_matches_oracle(B, T, heads, qk_scale):
+    need_cuda()
+    import vision_transformer_encoder_fwd_b200 as V
+    D = heads * 64
+    qkv = S.make_matrix((B, T, 3 * D), 10 + T, 1.0).float()
+    qkv[..., :2 * D] *= qk_scale
+    qkv = qkv.to(torch.bfloat16)
+    out, st = V.stage_attention(qkv.cuda(), heads)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    g = out.double().cpu().numpy()
+    r = _ref_attention(qkv, heads)
+    assert np.isfinite(g).all()
+    err = np.abs(g - r).max()
+    assert err <= 1e-2 * np.abs(r).max() + 2e-3, err
+
+
+def test_attention_huge_logits_stay_finite():
+    """kornia/dinov3 card, "Build BF16, not FP16": scaled logits of ~2e6 must not overflow."""
+    need_cuda()
+    import vision_transformer_encoder_fwd_b200 as V
+    B, T, heads = 1, 300, 1
+    D = 64
+    qkv = S.make_matrix((B, T, 3 * D), 99, 0.5).float()
+    # every query has 1500 on the first 8 dims; key 1 has 1470 there: logit 8*1500*1470/8 = 2.2e6
+    qkv[0, :, 0:8] = 1500.0
+    qkv[0, 1, D:D + 8] = 1470.0
+    qkv = qkv.to(torch.bfloat16)
+    out, st = V.stage_attention(qkv.cuda(), heads)
+    torch.cuda.synchronize()
+    g = out.double().cpu().numpy()
+    r = _ref_attention(qkv, heads)
+    assert np.isfinite(g).all() and int(st.item()) == 0
+    assert np.abs(g - r).max() <= 1e-2 * np.abs(r).max() + 2e-3
+    # the sink takes all the weight: every row equals v of key 1
+    assert np.abs(g[0] - qkv[0, 1, 2 * D:].double().numpy()).max() < 1e-2

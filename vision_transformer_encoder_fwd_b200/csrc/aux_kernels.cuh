@@ -1,0 +1,437 @@
+// Memory-bound kernels of the encoder forward and of the zero-shot scoring, plus the one-time
+// weight preparation run by vit_create.  None of these touches tensor cores: they are
+// HBM/L2-bound and laid out for coalesced 16-byte (or 4-byte per lane) accesses.
+#pragma once
+
+#include "common.cuh"
+
+namespace vit {
+
+// Source of the encoder's input pixels.  Image b of the batch is read at
+//   ptr[b * img_stride + c * chan_stride + (oy + y) * row_stride + (ox + x)]
+// with the window origin (oy, ox) of batch entry b = iy * nx + ix given by
+//   oy = min(iy * win_stride, max_oy), ox = min(ix * win_stride, max_ox)
+// (nx = 1, win_stride = 0 for a plain batch of images).
+struct ImgSrc {
+  const float* ptr;
+  long long img_stride, chan_stride, row_stride;
+  int nx, win_stride, max_oy, max_ox;
+};
+
+// kornia/dinov3 card "Model I/O" + "DINOv2 n semantic" diagram "Conv2d p x p / p": the
+// patch convolution as a GEMM needs A[b*P + p, k] = bf16(pixel), k = c*p^2 + ky*p + kx, zero
+// for k >= 3 p^2 up to Kpad.  Each thread writes 8 consecutive k (one 16-byte store).
+__global__ void im2col_bf16_kernel(ImgSrc src, int B, int p, int gw, int P, int Kpad, __nv_bfloat16* __restrict__ A) {
+  const int kv = Kpad / 8;
+  const long long total = static_cast<long long>(B) * P * kv;
+  const int pp = p * p;
+  const int K = 3 * pp;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int k8 = static_cast<int>(i % kv);
+    const long long row = i / kv;
+    const int b = static_cast<int>(row / P);
+    const int pi = static_cast<int>(row - static_cast<long long>(b) * P);
+    const int gy = pi / gw, gx = pi - gy * gw;
+    const int iy = b / src.nx, ix = b - iy * src.nx;
+    const int oy = min(iy * src.win_stride, src.max_oy) + gy * p;
+    const int ox = min(ix * src.win_stride, src.max_ox) + gx * p;
+    const float* base = src.ptr + b * src.img_stride;
+    float v[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int k = k8 * 8 + t;
+      float x = 0.f;
+      if (k < K) {
+        const int c = k / pp;
+        const int rem = k - c * pp;
+        const int ky = rem / p, kx = rem - ky * p;
+        x = __ldg(base + c * src.chan_stride + static_cast<long long>(oy + ky) * src.row_stride + (ox + kx));
+      }
+      v[t] = x;
+    }
+    uint4 w;
+    w.x = pack_bf16x2(v[0], v[1]);
+    w.y = pack_bf16x2(v[2], v[3]);
+    w.z = pack_bf16x2(v[4], v[5]);
+    w.w = pack_bf16x2(v[6], v[7]);
+    reinterpret_cast<uint4*>(A + row * Kpad)[k8] = w;
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// CLS and register rows of the residual stream ([card] "Model I/O": CLS, then 4 registers;
+// [diagram] position embedding row 0 on CLS for DINOv2): x, its bf16 copy and the per-group
+// (mean, M2) statistics the folded LayerNorm of block 1 reads.  grid (ngroups, 1 + R, B),
+// one warp per (row, column group of gcols).
+__global__ void prefix_tokens_kernel(const float* __restrict__ cls, const float* __restrict__ reg,
+                                     const float* __restrict__ pos, int pos_on_cls, int T, int D, int gcols,
+                                     float* __restrict__ x, __nv_bfloat16* __restrict__ xb, float2* __restrict__ stats) {
+  const int g = blockIdx.x, t = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x;
+  const size_t row = static_cast<size_t>(b) * T + t;
+  float s = 0.f;
+  for (int j = lane; j < gcols; j += 32) {
+    const int n = g * gcols + j;
+    float v = (t == 0) ? cls[n] + (pos_on_cls ? pos[n] : 0.f) : reg[static_cast<size_t>(t - 1) * D + n];
+    x[row * D + n] = v;
+    xb[row * D + n] = __float2bfloat16_rn(v);
+    s += v;
+  }
+  const float mean = warp_sum(s) / static_cast<float>(gcols);
+  float q = 0.f;
+  for (int j = lane; j < gcols; j += 32) {
+    const float d = x[row * D + g * gcols + j] - mean;
+    q = fmaf(d, d, q);
+  }
+  q = warp_sum(q);
+  if (lane == 0) stats[row * (D / gcols) + g] = make_float2(mean, q);
+}
+
+// Row LayerNorm statistics with one warp per row, two passes over the row (L1/L2-resident on
+// the second pass): biased variance, eps inside the square root ([diagram] "Encoder block").
+__device__ __forceinline__ void row_mean_rstd(const float* __restrict__ xr, int D, float eps, float& mean, float& rstd) {
+  const int lane = threadIdx.x & 31;
+  float s = 0.f;
+  for (int n = lane; n < D; n += 32) s += xr[n];
+  mean = warp_sum(s) / static_cast<float>(D);
+  float q = 0.f;
+  for (int n = lane; n < D; n += 32) {
+    const float d = xr[n] - mean;
+    q = fmaf(d, d, q);
+  }
+  q = warp_sum(q);
+  rstd = rsqrtf(q / static_cast<float>(D) + eps);
+}
+
+// Final LayerNorm and the encoder's outputs: the L2-normalised CLS descriptor ([card]
+// "Usage": "L2-normed [384], cosine-ready"; "Model I/O": descriptor = CLS token) and the
+// patch tokens (CLS and the R registers skipped, [card] "Model I/O").  One warp per
+// (image, token) with token 0 (CLS) or 1 + R .. T - 1 (patches).
+__global__ void final_ln_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ be,
+                                int B, int T, int R, int D, float eps, float* __restrict__ desc, void* __restrict__ patch,
+                                int patch_fp32) {
+  const int P = T - 1 - R;
+  const int warps_per_block = blockDim.x >> 5;
+  const long long job = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5);
+  const long long njobs = static_cast<long long>(B) * (1 + P);
+  if (job >= njobs) return;
+  const int lane = threadIdx.x & 31;
+  const int b = static_cast<int>(job / (1 + P));
+  const int j = static_cast<int>(job - static_cast<long long>(b) * (1 + P));
+  const int t = (j == 0) ? 0 : (j + R);
+  const float* xr = x + (static_cast<size_t>(b) * T + t) * D;
+  float mean, rstd;
+  row_mean_rstd(xr, D, eps, mean, rstd);
+  if (j == 0) {
+    if (desc == nullptr) return;
+    float q = 0.f;
+    for (int n = lane; n < D; n += 32) {
+      const float v = (xr[n] - mean) * rstd * g[n] + be[n];
+      q = fmaf(v, v, q);
+    }
+    q = warp_sum(q);
+    const float inv = 1.0f / fmaxf(sqrtf(q), 1e-12f);
+    for (int n = lane; n < D; n += 32) desc[static_cast<size_t>(b) * D + n] = ((xr[n] - mean) * rstd * g[n] + be[n]) * inv;
+  } else {
+    if (patch == nullptr) return;
+    const size_t o = (static_cast<size_t>(b) * P + (j - 1)) * D;
+    if (patch_fp32) {
+      float* dst = static_cast<float*>(patch) + o;
+      for (int n = lane; n < D; n += 32) dst[n] = (xr[n] - mean) * rstd * g[n] + be[n];
+    } else {
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(patch) + o;
+      for (int n = lane; n < D; n += 32) dst[n] = __float2bfloat16_rn((xr[n] - mean) * rstd * g[n] + be[n]);
+    }
+  }
+}
+
+// Taps ([diagram] "Tap stage l: 384 x 37 x 37"; "Taps apply LayerNorm, remove CLS, reshape"):
+// out[b, d, p] = LN_final(x[b, 1 + R + p])[d], channels first.  Block = 32 patches of one image:
+// 8 warps compute the 32 row statistics, then 32 x 32 tiles are transposed through shared
+// memory so that both the read (along d) and the write (along p) are coalesced.
+__global__ void tap_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ be, int T,
+                           int R, int D, float eps, float* __restrict__ out) {
+  __shared__ float tile[32][33];
+  __shared__ float s_mean[32], s_rstd[32];
+  const int P = T - 1 - R;
+  const int b = blockIdx.y;
+  const int p0 = blockIdx.x * 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = warp; i < 32; i += 8) {
+    const int p = p0 + i;
+    float mean = 0.f, rstd = 0.f;
+    if (p < P) row_mean_rstd(x + (static_cast<size_t>(b) * T + 1 + R + p) * D, D, eps, mean, rstd);
+    if (lane == 0) {
+      s_mean[i] = mean;
+      s_rstd[i] = rstd;
+    }
+  }
+  __syncthreads();
+  for (int d0 = 0; d0 < D; d0 += 32) {
+    for (int i = warp; i < 32; i += 8) {
+      const int p = p0 + i;
+      const int d = d0 + lane;
+      float v = 0.f;
+      if (p < P) v = (x[(static_cast<size_t>(b) * T + 1 + R + p) * D + d] - s_mean[i]) * s_rstd[i] * g[d] + be[d];
+      tile[i][lane] = v;
+    }
+    __syncthreads();
+    for (int i = warp; i < 32; i += 8) {
+      const int d = d0 + i;
+      const int p = p0 + lane;
+      if (p < P) out[(static_cast<size_t>(b) * D + d) * P + p] = tile[lane][i];
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ weight preparation
+// LayerNorm folded into the following Linear (exact algebra, gamma/beta of the LayerNorm,
+// W [N, K] of the Linear):
+//   LN(x) W^T + b = rstd * (x Wg^T - mean * colsum(Wg)) + (b + W beta),  Wg[n, k] = gamma_k W[n, k]
+// This kernel writes Wg in bf16, colsum over the bf16 Wg (so the mean term cancels the
+// operand the MMA actually multiplies) and the folded bias in fp32.  One block per row n.
+__global__ void fold_ln_weight_kernel(const __nv_bfloat16* __restrict__ W, const __nv_bfloat16* __restrict__ bias,
+                                      const __nv_bfloat16* __restrict__ gamma, const __nv_bfloat16* __restrict__ beta,
+                                      int N, int K, __nv_bfloat16* __restrict__ Wg, float* __restrict__ colsum,
+                                      float* __restrict__ bias_out) {
+  __shared__ double red[2][32];
+  const int n = blockIdx.x;
+  double cs = 0.0, bb = 0.0;
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    const float w = __bfloat162float(W[static_cast<size_t>(n) * K + k]);
+    const __nv_bfloat16 wg = __float2bfloat16_rn(w * __bfloat162float(gamma[k]));
+    Wg[static_cast<size_t>(n) * K + k] = wg;
+    cs += static_cast<double>(__bfloat162float(wg));
+    bb += static_cast<double>(w) * static_cast<double>(__bfloat162float(beta[k]));
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    cs += __shfl_xor_sync(0xffffffffu, cs, o);
+    bb += __shfl_xor_sync(0xffffffffu, bb, o);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    red[0][warp] = cs;
+    red[1][warp] = bb;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double a = 0.0, c = 0.0;
+    for (int w = 0; w < (blockDim.x >> 5); ++w) {
+      a += red[0][w];
+      c += red[1][w];
+    }
+    colsum[n] = static_cast<float>(a);
+    bias_out[n] = static_cast<float>(static_cast<double>(__bfloat162float(bias[n])) + c);
+  }
+}
+
+// Patch-embedding weight [D, 3 p^2] copied into [D, Kpad] with zero columns past 3 p^2.
+__global__ void pad_rows_bf16_kernel(const __nv_bfloat16* __restrict__ src, int rows, int K, int Kpad,
+                                     __nv_bfloat16* __restrict__ dst) {
+  const long long total = static_cast<long long>(rows) * Kpad;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / Kpad;
+    const int k = static_cast<int>(i - r * Kpad);
+    dst[i] = (k < K) ? src[r * K + k] : __float2bfloat16_rn(0.f);
+  }
+}
+
+__global__ void bf16_to_f32_kernel(const __nv_bfloat16* __restrict__ src, long long n, float* __restrict__ dst) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    dst[i] = __bfloat162float(src[i]);
+}
+
+// ------------------------------------------------------------------ zero-shot scoring
+// dino.txt article, patch/text alignment: F.normalize of each patch token, then
+// einsum("cd,hwd->chw") with the text features.  Step 1: inv_norm[i] = 1 / max(||t_i||, 1e-12),
+// one warp per token.
+__global__ void token_inv_norm_kernel(const float* __restrict__ tok, long long rows, int D, float* __restrict__ inv) {
+  const long long r = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const int lane = threadIdx.x & 31;
+  float q = 0.f;
+  for (int n = lane; n < D; n += 32) {
+    const float v = tok[r * D + n];
+    q = fmaf(v, v, q);
+  }
+  q = warp_sum(q);
+  if (lane == 0) inv[r] = 1.0f / fmaxf(sqrtf(q), 1e-12f);
+}
+
+// Step 2: cos[w, c, i] = inv[w, i] * sum_d text[c, d] tok[w, i, d], an fp32 SIMT GEMM tile of
+// 64 tokens x 64 classes per block (16 x 16 threads, 4 x 4 outputs each, K staged by 16).
+// fp32 keeps the class ranking exact enough for the argmax (scores differ by ~1e-2).
+__global__ void cos_gemm_kernel(const float* __restrict__ tok, const float* __restrict__ inv,
+                                const float* __restrict__ text, int rows_per_win, long long rows, int C, int D,
+                                float* __restrict__ cosout) {
+  __shared__ float sa[16][64 + 4];
+  __shared__ float sb[16][64 + 4];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const long long r0 = static_cast<long long>(blockIdx.x) * 64;
+  const int c0 = blockIdx.y * 64;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < D; k0 += 16) {
+    for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+      const int rr = i >> 4, kk = i & 15;
+      const long long r = r0 + rr;
+      sa[kk][rr] = (r < rows) ? tok[r * D + k0 + kk] : 0.f;
+      const int c = c0 + rr;
+      sb[kk][rr] = (c < C) ? text[static_cast<size_t>(c) * D + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = sa[kk][ty * 4 + i];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) bv[i] = sb[kk][tx * 4 + i];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) acc[i][jj] = fmaf(a[i], bv[jj], acc[i][jj]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const long long r = r0 + ty * 4 + i;
+    if (r >= rows) continue;
+    const long long w = r / rows_per_win;
+    const long long pi = r - w * rows_per_win;
+    const float s = inv[r];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int c = c0 + tx * 4 + jj;
+      if (c < C) cosout[(w * C + c) * rows_per_win + pi] = acc[i][jj] * s;
+    }
+  }
+}
+
+// Bilinear source taps of output index i for an in -> out resize with align_corners=False:
+// src = (i + 0.5) * in / out - 0.5 clamped below at 0; neighbours floor(src) and
+// min(floor + 1, in - 1); weight of the upper one = fractional part.
+struct Taps1D {
+  int i0, i1;
+  float w1;
+};
+__device__ __forceinline__ Taps1D bilinear_taps(int i, int n_in, int n_out) {
+  float src = (static_cast<float>(i) + 0.5f) * (static_cast<float>(n_in) / static_cast<float>(n_out)) - 0.5f;
+  src = fmaxf(src, 0.f);
+  int i0 = min(static_cast<int>(src), n_in - 1);
+  Taps1D t;
+  t.i0 = i0;
+  t.i1 = min(i0 + 1, n_in - 1);
+  t.w1 = src - static_cast<float>(i0);
+  return t;
+}
+
+// Slide mode (dino.txt article, whole/slide section): for every pixel, the windows covering it
+// (at most 6 here) each contribute softmax_c(bilinear(cos_w)) and the sum is divided by the
+// covering count; label = argmax_c (lowest index on ties).  Gather form: each thread owns one
+// pixel and visits its windows, so probs is written exactly once and no atomics are needed.
+__global__ void seg_slide_kernel(const float* __restrict__ cosm, int C, int g, int H, int W, int side, int stride, int ny,
+                                 int nx, float* __restrict__ probs, int* __restrict__ labels) {
+  const long long pix = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (pix >= static_cast<long long>(H) * W) return;
+  const int y = static_cast<int>(pix / W), x = static_cast<int>(pix - static_cast<long long>(y) * W);
+  constexpr int MAXW = 16;
+  int off[MAXW][4];
+  float wt[MAXW][4];
+  int nw = 0;
+  for (int iy = 0; iy < ny; ++iy) {
+    const int oy = min(iy * stride, H - side);
+    if (y < oy || y >= oy + side) continue;
+    const Taps1D ty = bilinear_taps(y - oy, g, side);
+    for (int ix = 0; ix < nx; ++ix) {
+      const int ox = min(ix * stride, W - side);
+      if (x < ox || x >= ox + side || nw >= MAXW) continue;
+      const Taps1D tx = bilinear_taps(x - ox, g, side);
+      const int base = (iy * nx + ix) * C * g * g;
+      off[nw][0] = base + ty.i0 * g + tx.i0;
+      off[nw][1] = base + ty.i0 * g + tx.i1;
+      off[nw][2] = base + ty.i1 * g + tx.i0;
+      off[nw][3] = base + ty.i1 * g + tx.i1;
+      wt[nw][0] = (1.f - ty.w1) * (1.f - tx.w1);
+      wt[nw][1] = (1.f - ty.w1) * tx.w1;
+      wt[nw][2] = ty.w1 * (1.f - tx.w1);
+      wt[nw][3] = ty.w1 * tx.w1;
+      ++nw;
+    }
+  }
+  const int gg = g * g;
+  float mx[MAXW], inv_sum[MAXW];
+  for (int w = 0; w < nw; ++w) {
+    float m = -INFINITY;
+    for (int c = 0; c < C; ++c) {
+      const float* cm = cosm + c * gg;
+      const float v = wt[w][0] * __ldg(cm + off[w][0]) + wt[w][1] * __ldg(cm + off[w][1]) +
+                      wt[w][2] * __ldg(cm + off[w][2]) + wt[w][3] * __ldg(cm + off[w][3]);
+      m = fmaxf(m, v);
+    }
+    float s = 0.f;
+    for (int c = 0; c < C; ++c) {
+      const float* cm = cosm + c * gg;
+      const float v = wt[w][0] * __ldg(cm + off[w][0]) + wt[w][1] * __ldg(cm + off[w][1]) +
+                      wt[w][2] * __ldg(cm + off[w][2]) + wt[w][3] * __ldg(cm + off[w][3]);
+      s += expf(v - m);
+    }
+    mx[w] = m;
+    inv_sum[w] = 1.0f / s;
+  }
+  const float inv_count = 1.0f / static_cast<float>(nw);
+  float best = -INFINITY;
+  int best_c = 0;
+  for (int c = 0; c < C; ++c) {
+    const float* cm = cosm + c * gg;
+    float p = 0.f;
+    for (int w = 0; w < nw; ++w) {
+      const float v = wt[w][0] * __ldg(cm + off[w][0]) + wt[w][1] * __ldg(cm + off[w][1]) +
+                      wt[w][2] * __ldg(cm + off[w][2]) + wt[w][3] * __ldg(cm + off[w][3]);
+      p += expf(v - mx[w]) * inv_sum[w];
+    }
+    p *= inv_count;
+    if (probs) probs[static_cast<size_t>(c) * H * W + pix] = p;
+    if (p > best) {
+      best = p;
+      best_c = c;
+    }
+  }
+  if (labels) labels[pix] = best_c;
+}
+
+// Whole mode: scores = bilinear upsample of the cosine map [C, gh, gw] to [C, H, W]; argmax.
+__global__ void seg_whole_kernel(const float* __restrict__ cosm, int C, int gh, int gw, int H, int W,
+                                 float* __restrict__ scores, int* __restrict__ labels) {
+  const long long pix = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (pix >= static_cast<long long>(H) * W) return;
+  const int y = static_cast<int>(pix / W), x = static_cast<int>(pix - static_cast<long long>(y) * W);
+  const Taps1D ty = bilinear_taps(y, gh, H);
+  const Taps1D tx = bilinear_taps(x, gw, W);
+  const float w00 = (1.f - ty.w1) * (1.f - tx.w1), w01 = (1.f - ty.w1) * tx.w1;
+  const float w10 = ty.w1 * (1.f - tx.w1), w11 = ty.w1 * tx.w1;
+  float best = -INFINITY;
+  int best_c = 0;
+  for (int c = 0; c < C; ++c) {
+    const float* cm = cosm + static_cast<size_t>(c) * gh * gw;
+    const float v = w00 * __ldg(cm + ty.i0 * gw + tx.i0) + w01 * __ldg(cm + ty.i0 * gw + tx.i1) +
+                    w10 * __ldg(cm + ty.i1 * gw + tx.i0) + w11 * __ldg(cm + ty.i1 * gw + tx.i1);
+    if (scores) scores[static_cast<size_t>(c) * H * W + pix] = v;
+    if (v > best) {
+      best = v;
+      best_c = c;
+    }
+  }
+  if (labels) labels[pix] = best_c;
+}
+
+}  // namespace vit

@@ -1,0 +1,356 @@
+// Persistent tcgen05 GEMM for sm_100a: C[M, N] = A[M, K] . B[N, K]^T with bf16 operands
+// (both K-contiguous, nn.Linear layout for B) and an fp32 accumulator in tensor memory,
+// followed by one of the encoder's fused epilogues.
+//
+// CTA = 6 warps, one CTA per SM, grid = min(#tiles, #SMs), tiles visited with stride gridDim:
+//   warp 0 (one lane)  TMA producer: A tile 128 x 64 and B tile BN x 64 per stage, 128-byte
+//                      swizzle, STAGES-deep ring guarded by full/empty mbarriers.
+//   warp 1             allocates 512 TMEM columns (two BN-wide fp32 accumulators); one lane
+//                      issues tcgen05.mma (M = 128, N = BN, K = 16) four times per stage and
+//                      commits each stage back to the producer and each finished tile to
+//                      the epilogue.
+//   warps 2..5         epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, i.e. one output
+//                      row per thread, 32 columns per tcgen05.ld; applies the epilogue and
+//                      writes global memory, then releases the accumulator.
+// The double-buffered accumulator lets the epilogue of tile i overlap the MMAs of tile i+1.
+#pragma once
+
+#include "common.cuh"
+
+namespace vit {
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BK = 64;
+constexpr int GEMM_THREADS = 192;
+
+enum EpiMode : int {
+  EPI_BIAS = 0,    // out_bf16 = act(acc + bias)
+  EPI_LNFOLD = 1,  // out_bf16 = act(rstd * (acc - mean * colsum) + bias)  (LayerNorm folded)
+  EPI_RESID = 2,   // x += ls * (acc + bias); xb = bf16(x); row partial stats of x
+  EPI_PATCH = 3,   // x[token row] = acc + bias + pos; xb; row partial stats
+};
+
+struct EpiParams {
+  int M, N;
+  const float* bias;  // [N]
+  int gelu;           // BIAS / LNFOLD: apply exact-erf GELU
+  __nv_bfloat16* out;  // BIAS / LNFOLD output [M, ldo]
+  int ldo;
+  // LNFOLD: per-row LayerNorm statistics rebuilt from partials written by the producer of x
+  const float* colsum;     // [N] column sums of the gamma-folded weight
+  const float2* stats_in;  // [M, nt] (mean, M2) of column groups of nt_cols each
+  int nt, nt_cols, D;
+  float eps;
+  // RESID / PATCH
+  float* x;              // [rows, N] fp32 residual stream
+  __nv_bfloat16* xb;     // [rows, N] bf16 copy of x (A operand of the next folded GEMM)
+  const float* ls;       // [N] layer scale (RESID)
+  float2* stats_out;     // [rows, N / BN] (mean, M2) over each BN-column group
+  // PATCH: GEMM row m = b * P + p goes to token row b * T + 1 + R + p, position row p + pos_off
+  const float* pos;
+  int P, T, R, pos_off;
+};
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
+  static constexpr int B_BYTES = BN * GEMM_BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+  static constexpr uint32_t TMEM_COLS = 512;
+};
+
+__device__ __forceinline__ void merge_stats(float& n, float& mean, float& m2, float nb, float mb, float m2b) {
+  const float tot = n + nb;
+  const float d = mb - mean;
+  mean += d * (nb / tot);
+  m2 += m2b + d * d * (n * nb / tot);
+  n = tot;
+}
+
+template <int BN, int MODE>
+__device__ __forceinline__ void gemm_epilogue_tile(const EpiParams& ep, uint32_t taddr, int row, int n0) {
+  const bool valid = row < ep.M;
+  float mu = 0.f, rstd = 0.f;
+  if (MODE == EPI_LNFOLD && valid) {
+    float n = 0.f, mean = 0.f, m2 = 0.f;
+    const float2* s = ep.stats_in + static_cast<size_t>(row) * ep.nt;
+    for (int t = 0; t < ep.nt; ++t) {
+      const float2 st = s[t];
+      merge_stats(n, mean, m2, static_cast<float>(ep.nt_cols), st.x, st.y);
+    }
+    mu = mean;
+    rstd = rsqrtf(m2 / static_cast<float>(ep.D) + ep.eps);
+  }
+  int xrow = row;
+  const float* posrow = nullptr;
+  if (MODE == EPI_PATCH && valid) {
+    const int b = row / ep.P;
+    const int p = row - b * ep.P;
+    xrow = b * ep.T + 1 + ep.R + p;
+    posrow = ep.pos + static_cast<size_t>(p + ep.pos_off) * ep.N;
+  }
+  float run_n = 0.f, run_mean = 0.f, run_m2 = 0.f;
+
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    float v[32];
+    __syncwarp();
+    tmem_ld32(taddr + c * 32, v);
+    const int n = n0 + c * 32;
+    if (valid) {
+      if (MODE == EPI_BIAS || MODE == EPI_LNFOLD) {
+        const float4* b4 = reinterpret_cast<const float4*>(ep.bias + n);
+        if (MODE == EPI_LNFOLD) {
+          const float4* c4 = reinterpret_cast<const float4*>(ep.colsum + n);
+          const float rm = rstd * mu;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 bb = __ldg(b4 + j);
+            const float4 cc = __ldg(c4 + j);
+            v[4 * j + 0] = fmaf(rstd, v[4 * j + 0], fmaf(-rm, cc.x, bb.x));
+            v[4 * j + 1] = fmaf(rstd, v[4 * j + 1], fmaf(-rm, cc.y, bb.y));
+            v[4 * j + 2] = fmaf(rstd, v[4 * j + 2], fmaf(-rm, cc.z, bb.z));
+            v[4 * j + 3] = fmaf(rstd, v[4 * j + 3], fmaf(-rm, cc.w, bb.w));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 bb = __ldg(b4 + j);
+            v[4 * j + 0] += bb.x;
+            v[4 * j + 1] += bb.y;
+            v[4 * j + 2] += bb.z;
+            v[4 * j + 3] += bb.w;
+          }
+        }
+        if (ep.gelu) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+        }
+        uint4* o = reinterpret_cast<uint4*>(ep.out + static_cast<size_t>(row) * ep.ldo + n);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 w;
+          w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+          w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+          w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+          w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+          o[j] = w;
+        }
+      } else {
+        float4* xp = reinterpret_cast<float4*>(ep.x + static_cast<size_t>(xrow) * ep.N + n);
+        const float4* b4 = reinterpret_cast<const float4*>(ep.bias + n);
+        if (MODE == EPI_RESID) {
+          const float4* l4 = reinterpret_cast<const float4*>(ep.ls + n);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 xo = xp[j];
+            const float4 bb = __ldg(b4 + j);
+            const float4 ll = __ldg(l4 + j);
+            v[4 * j + 0] = fmaf(ll.x, v[4 * j + 0] + bb.x, xo.x);
+            v[4 * j + 1] = fmaf(ll.y, v[4 * j + 1] + bb.y, xo.y);
+            v[4 * j + 2] = fmaf(ll.z, v[4 * j + 2] + bb.z, xo.z);
+            v[4 * j + 3] = fmaf(ll.w, v[4 * j + 3] + bb.w, xo.w);
+          }
+        } else {
+          const float4* p4 = reinterpret_cast<const float4*>(posrow + n);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 bb = __ldg(b4 + j);
+            const float4 pp = __ldg(p4 + j);
+            v[4 * j + 0] += bb.x + pp.x;
+            v[4 * j + 1] += bb.y + pp.y;
+            v[4 * j + 2] += bb.z + pp.z;
+            v[4 * j + 3] += bb.w + pp.w;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xp[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        uint4* o = reinterpret_cast<uint4*>(ep.xb + static_cast<size_t>(xrow) * ep.N + n);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 w;
+          w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+          w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+          w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+          w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+          o[j] = w;
+        }
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s += v[j];
+        const float cm = s * (1.0f / 32.0f);
+        float q = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float d = v[j] - cm;
+          q = fmaf(d, d, q);
+        }
+        merge_stats(run_n, run_mean, run_m2, 32.f, cm, q);
+      }
+    }
+  }
+  if ((MODE == EPI_RESID || MODE == EPI_PATCH) && valid) {
+    ep.stats_out[static_cast<size_t>(xrow) * (ep.N / BN) + n0 / BN] = make_float2(run_mean, run_m2);
+  }
+}
+
+template <int BN, int MODE>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
+                        int N, int K, EpiParams ep, int* gstatus) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = (*reinterpret_cast<volatile int*>(gstatus) != 0) ? 1 : 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const bool skip = *abort_flag != 0;
+
+  const int num_m = (M + GEMM_BM - 1) / GEMM_BM;
+  const int num_n = N / BN;
+  const int num_tiles = num_m * num_n;
+  const int KB = K / GEMM_BK;
+
+  if (!skip && warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued_parity[STAGES];
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int mb = tile / num_n;
+      const int nb = tile - mb * num_n;
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+        tma_load_2d(sA + stage * Cfg::A_BYTES, &tmA, kb * GEMM_BK, mb * GEMM_BM, &full[stage]);
+        tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, kb * GEMM_BK, nb * BN, &full[stage]);
+        issued_parity[stage] = static_cast<int>(phase);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+    }
+    if (*abort_flag) {
+      // let every issued tile land before the CTA can exit and release its shared memory
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_parity[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(issued_parity[s]));
+    }
+  } else if (!skip && warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(GEMM_BM, BN, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 2)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * Cfg::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < GEMM_BK / 16; ++k) {
+            tc_mma_ss(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024), sdesc_sw128(b0 + k * 32, 16, 1024), idesc,
+                      (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      tc_commit(mma_done);
+    }
+    __syncwarp();
+  } else if (!skip && warp >= 2) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int mb = tile / num_n;
+      const int nb = tile - mb * num_n;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 4)) break;
+      tc_fence_after();
+      const int row = mb * GEMM_BM + q * 32 + lane;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      gemm_epilogue_tile<BN, MODE>(ep, taddr, row, nb * BN);
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  __syncthreads();
+  if (warp == 1) {
+    if (!skip && lane == 0) {
+      // all MMAs issued by this CTA have completed before TMEM is released
+      mbar_wait_drain(mma_done, 0);
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace vit

@@ -1,0 +1,939 @@
+// libvit_b200: host side of the C ABI declared in include/vit.h and include/vit_stages.h.
+//
+// Plans and launches the encoder forward of the DINOv2/DINOv3 ViT ("DINOv2 n semantic"
+// diagram; kornia/dinov3 card) and the dino.txt zero-shot scoring on one B200:
+//   im2col -> patch GEMM (+bias +pos, token placement, row stats) -> CLS/register rows
+//   per block: QKV GEMM (LayerNorm folded) -> attention -> proj GEMM (+LS, residual, stats)
+//              -> FC1 GEMM (LayerNorm folded, GELU) -> FC2 GEMM (+LS, residual, stats) [-> tap]
+//   final LayerNorm -> descriptor / patch tokens
+// All compute runs in the kernels of this library; this file only validates, lays out the
+// workspace, encodes TMA descriptors and enqueues launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/vit.h"
+#include "../../include/vit_stages.h"
+#include "attention.cuh"
+#include "aux_kernels.cuh"
+#include "gemm.cuh"
+
+using namespace vit;
+
+namespace {
+
+thread_local std::string g_err;
+
+void set_err(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+}
+
+#define CK(call)                                                                              \
+  do {                                                                                        \
+    cudaError_t e_ = (call);                                                                  \
+    if (e_ != cudaSuccess) {                                                                  \
+      set_err("%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), __FILE__, __LINE__);     \
+      return VIT_E_CUDA;                                                                      \
+    }                                                                                         \
+  } while (0)
+
+#define CKL()                                                                                 \
+  do {                                                                                        \
+    cudaError_t e_ = cudaGetLastError();                                                      \
+    if (e_ != cudaSuccess) {                                                                  \
+      set_err("kernel launch failed: %s (%s:%d)", cudaGetErrorString(e_), __FILE__, __LINE__); \
+      return VIT_E_CUDA;                                                                      \
+    }                                                                                         \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ TMA descriptor encoding
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [rows, cols] matrix with leading dimension ld (elements);
+// box = box_cols x box_rows with box_cols * 2 bytes == 128 (one 128-byte swizzle row).
+bool tmap_2d(CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_cols,
+             uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    set_err("cuTensorMapEncodeTiled is not available from the driver");
+    return false;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_err("cuTensorMapEncodeTiled(2d) failed with %d (cols %llu rows %llu ld %llu)", static_cast<int>(r),
+            static_cast<unsigned long long>(cols), static_cast<unsigned long long>(rows),
+            static_cast<unsigned long long>(ld));
+    return false;
+  }
+  return true;
+}
+
+// 3-D bf16 map over qkv [B, T, 3D]: dims {3D, T, B}, box {64, 128, 1}.
+bool tmap_qkv3d(CUtensorMap* tm, const void* base, int B, int T, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    set_err("cuTensorMapEncodeTiled is not available from the driver");
+    return false;
+  }
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(3 * D), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(3 * D) * 2, static_cast<cuuint64_t>(T) * 3 * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(ATT_BM), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_err("cuTensorMapEncodeTiled(3d) failed with %d", static_cast<int>(r));
+    return false;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ launch helpers
+int device_sms(int dev) {
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 1;
+}
+
+template <typename K>
+cudaError_t set_smem_attr_once(K kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load() & bit) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit);
+  return e;
+}
+
+template <int BN, int MODE>
+cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, const EpiParams& ep,
+                          int* st, cudaStream_t s, int nsm) {
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t e = set_smem_attr_once(gemm_bf16_tc_kernel<BN, MODE>, GemmCfg<BN>::SMEM_BYTES, attr_done);
+  if (e != cudaSuccess) return e;
+  const int tiles = ((M + GEMM_BM - 1) / GEMM_BM) * (N / BN);
+  const int grid = std::max(1, std::min(tiles, nsm));
+  gemm_bf16_tc_kernel<BN, MODE><<<grid, GEMM_THREADS, GemmCfg<BN>::SMEM_BYTES, s>>>(a, b, M, N, K, ep, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(int bn, int mode, const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
+                        const EpiParams& ep, int* st, cudaStream_t s, int nsm) {
+  if (bn == 256) {
+    switch (mode) {
+      case EPI_BIAS: return launch_gemm_t<256, EPI_BIAS>(a, b, M, N, K, ep, st, s, nsm);
+      case EPI_LNFOLD: return launch_gemm_t<256, EPI_LNFOLD>(a, b, M, N, K, ep, st, s, nsm);
+      case EPI_RESID: return launch_gemm_t<256, EPI_RESID>(a, b, M, N, K, ep, st, s, nsm);
+      default: return launch_gemm_t<256, EPI_PATCH>(a, b, M, N, K, ep, st, s, nsm);
+    }
+  }
+  switch (mode) {
+    case EPI_BIAS: return launch_gemm_t<128, EPI_BIAS>(a, b, M, N, K, ep, st, s, nsm);
+    case EPI_LNFOLD: return launch_gemm_t<128, EPI_LNFOLD>(a, b, M, N, K, ep, st, s, nsm);
+    case EPI_RESID: return launch_gemm_t<128, EPI_RESID>(a, b, M, N, K, ep, st, s, nsm);
+    default: return launch_gemm_t<128, EPI_PATCH>(a, b, M, N, K, ep, st, s, nsm);
+  }
+}
+
+cudaError_t launch_attention(const CUtensorMap& tm, int B, int T, int heads, __nv_bfloat16* out, int* st,
+                             cudaStream_t s) {
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel, AttnCfg::SMEM_BYTES, attr_done);
+  if (e != cudaSuccess) return e;
+  dim3 grid((T + ATT_BM - 1) / ATT_BM, heads, B);
+  attn_fwd_tc_kernel<<<grid, ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, T, heads * 64, out, st);
+  return cudaGetLastError();
+}
+
+int grid_1d(long long work, int block, int nsm) {
+  long long g = (work + block - 1) / block;
+  return static_cast<int>(std::max(1LL, std::min(g, static_cast<long long>(nsm) * 32)));
+}
+
+// GEMM N-tile: 256 columns when N allows it and the tile count still fills the SMs.
+int pick_bn(int M, int N, int nsm) {
+  if (N % 256 != 0) return 128;
+  const long long tiles256 = static_cast<long long>((M + GEMM_BM - 1) / GEMM_BM) * (N / 256);
+  return tiles256 >= nsm ? 256 : 128;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ model
+struct BlockW {
+  __nv_bfloat16* qkv_wg;  // [3D, D] gamma-folded (owned)
+  float* qkv_c;           // [3D]
+  float* qkv_b;           // [3D] beta-folded bias
+  const __nv_bfloat16* proj_w;  // borrowed
+  float* proj_b;
+  float* ls1;
+  __nv_bfloat16* fc1_wg;  // [F, D] (owned)
+  float* fc1_c;
+  float* fc1_b;
+  const __nv_bfloat16* fc2_w;  // borrowed
+  float* fc2_b;
+  float* ls2;
+  CUtensorMap tm_qkv[2], tm_fc1[2];  // [0]: box rows 128, [1]: 256
+  CUtensorMap tm_proj, tm_fc2;       // box rows bn_res
+};
+
+struct vit_model {
+  vit_config cfg;
+  int device = 0, nsm = 1;
+  int gh = 0, gw = 0, P = 0, T = 0, K_pe = 0, Kpad = 0, bn_res = 128, nt = 1;
+  __nv_bfloat16* patch_w = nullptr;  // [D, Kpad]
+  float *patch_b = nullptr, *pos = nullptr, *cls = nullptr, *reg = nullptr, *norm_w = nullptr, *norm_b = nullptr;
+  CUtensorMap tm_patch;
+  std::vector<BlockW> blocks;
+  int* d_status = nullptr;
+  int last_launches = 0;
+  std::vector<void*> allocs;
+  // per-launch profiling (vit_profile_begin / vit_profile_end)
+  bool prof_on = false;
+  std::vector<cudaEvent_t> prof_ev;  // 2 per slot
+  std::vector<int> prof_kind;
+  int prof_used = 0;
+};
+
+namespace {
+
+struct WsLayout {
+  size_t x, xb, stats, attn, big, total;
+};
+
+WsLayout ws_layout(const vit_model* m, int B) {
+  const size_t M = static_cast<size_t>(B) * m->T, Mp = static_cast<size_t>(B) * m->P;
+  const size_t D = m->cfg.dim, F = m->cfg.mlp_dim;
+  WsLayout L;
+  size_t off = 0;
+  L.x = off;
+  off = align_up(off + M * D * 4, 1024);
+  L.xb = off;
+  off = align_up(off + M * D * 2, 1024);
+  L.stats = off;
+  off = align_up(off + M * m->nt * 8, 1024);
+  L.attn = off;
+  off = align_up(off + M * D * 2, 1024);
+  L.big = off;
+  off = align_up(off + std::max(std::max(M * 3 * D, M * F), Mp * static_cast<size_t>(m->Kpad)) * 2, 1024);
+  L.total = off;
+  return L;
+}
+
+// Profiling brackets around one launch (no-ops unless profiling is on and capacity remains).
+int prof_open(vit_model* m, int kind, cudaStream_t s) {
+  if (!m->prof_on || m->prof_used >= static_cast<int>(m->prof_kind.size())) return -1;
+  const int slot = m->prof_used++;
+  m->prof_kind[slot] = kind;
+  cudaEventRecord(m->prof_ev[2 * slot], s);
+  return slot;
+}
+void prof_close(vit_model* m, int slot, cudaStream_t s) {
+  if (slot >= 0) cudaEventRecord(m->prof_ev[2 * slot + 1], s);
+}
+
+vit_status alloc_dev(vit_model* m, void** p, size_t bytes) {
+  CK(cudaMalloc(p, std::max<size_t>(bytes, 16)));
+  m->allocs.push_back(*p);
+  return VIT_OK;
+}
+
+vit_status to_f32(vit_model* m, const void* src, size_t n, float** dst, cudaStream_t s) {
+  vit_status st = alloc_dev(m, reinterpret_cast<void**>(dst), n * 4);
+  if (st != VIT_OK) return st;
+  if (n == 0) return VIT_OK;
+  bf16_to_f32_kernel<<<grid_1d(static_cast<long long>(n), 256, m->nsm), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(src), static_cast<long long>(n), *dst);
+  CKL();
+  return VIT_OK;
+}
+
+vit_status validate_cfg(const vit_config* c) {
+  if (!c) {
+    set_err("config is NULL");
+    return VIT_E_INVALID_ARG;
+  }
+  if (c->heads < 1 || c->dim != c->heads * 64) {
+    set_err("dim (%d) must equal heads (%d) * 64", c->dim, c->heads);
+    return VIT_E_UNSUPPORTED;
+  }
+  if (c->dim % 128 != 0 || c->mlp_dim % 128 != 0 || c->mlp_dim < 128) {
+    set_err("dim (%d) and mlp_dim (%d) must be multiples of 128", c->dim, c->mlp_dim);
+    return VIT_E_UNSUPPORTED;
+  }
+  if (c->patch < 1 || c->patch > 32 || c->img_h < c->patch || c->img_w < c->patch || c->img_h % c->patch ||
+      c->img_w % c->patch) {
+    set_err("image %dx%d must be a positive multiple of patch %d (1..32)", c->img_h, c->img_w, c->patch);
+    return VIT_E_SHAPE;
+  }
+  if (c->n_registers < 0 || c->n_registers > 16 || c->depth < 1 || c->depth > 64 || c->max_batch < 1 ||
+      !(c->ln_eps > 0.f)) {
+    set_err("n_registers 0..16, depth 1..64, max_batch >= 1 and ln_eps > 0 required");
+    return VIT_E_INVALID_ARG;
+  }
+  int ntaps = 0;
+  for (int l = 0; l < 32; ++l)
+    if (c->tap_mask & (1u << l)) {
+      ++ntaps;
+      if (l + 1 > c->depth) {
+        set_err("tap after block %d exceeds depth %d", l + 1, c->depth);
+        return VIT_E_INVALID_ARG;
+      }
+    }
+  if (ntaps > 4) {
+    set_err("at most 4 taps");
+    return VIT_E_INVALID_ARG;
+  }
+  return VIT_OK;
+}
+
+struct Scratch {
+  float* x;
+  __nv_bfloat16* xb;
+  float2* stats;
+  __nv_bfloat16* attn;
+  __nv_bfloat16* big;
+};
+
+// The encoder forward on B images read through `src`; outputs per `out`.
+vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs* out, void* ws, size_t ws_bytes,
+                       cudaStream_t s) {
+  const vit_config& c = m->cfg;
+  const WsLayout L = ws_layout(m, B);
+  if (ws == nullptr || ws_bytes < L.total) {
+    set_err("workspace of %zu bytes is smaller than the %zu required for batch %d", ws_bytes, L.total, B);
+    return VIT_E_WORKSPACE;
+  }
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) {
+    set_err("workspace must be 256-byte aligned");
+    return VIT_E_INVALID_ARG;
+  }
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  Scratch S{reinterpret_cast<float*>(w8 + L.x), reinterpret_cast<__nv_bfloat16*>(w8 + L.xb),
+            reinterpret_cast<float2*>(w8 + L.stats), reinterpret_cast<__nv_bfloat16*>(w8 + L.attn),
+            reinterpret_cast<__nv_bfloat16*>(w8 + L.big)};
+  const int D = c.dim, F = c.mlp_dim, T = m->T, P = m->P, R = c.n_registers;
+  const int M = B * T, Mp = B * P;
+  int launches = 0;
+
+  CUtensorMap tm_pe, tm_xb, tm_attn, tm_h, tm_qkv3;
+  if (!tmap_2d(&tm_pe, S.big, m->Kpad, Mp, m->Kpad, 64, GEMM_BM) || !tmap_2d(&tm_xb, S.xb, D, M, D, 64, GEMM_BM) ||
+      !tmap_2d(&tm_attn, S.attn, D, M, D, 64, GEMM_BM) || !tmap_2d(&tm_h, S.big, F, M, F, 64, GEMM_BM) ||
+      !tmap_qkv3d(&tm_qkv3, S.big, B, T, D))
+    return VIT_E_CUDA;
+
+  // patch embedding: im2col, GEMM with bias + position embedding, token placement
+  { const int ps_ = prof_open(m, VIT_K_IM2COL, s);
+  im2col_bf16_kernel<<<grid_1d(static_cast<long long>(Mp) * (m->Kpad / 8), 256, m->nsm), 256, 0, s>>>(
+      src, B, c.patch, m->gw, P, m->Kpad, S.big);
+  prof_close(m, ps_, s); }
+  CKL();
+  ++launches;
+  {
+    EpiParams ep{};
+    ep.M = Mp;
+    ep.N = D;
+    ep.bias = m->patch_b;
+    ep.x = S.x;
+    ep.xb = S.xb;
+    ep.stats_out = S.stats;
+    ep.pos = m->pos;
+    ep.P = P;
+    ep.T = T;
+    ep.R = R;
+    ep.pos_off = c.pos_on_cls ? 1 : 0;
+    { const int ps_ = prof_open(m, VIT_K_PATCH_GEMM, s);
+    CK(launch_gemm(m->bn_res, EPI_PATCH, tm_pe, m->tm_patch, Mp, D, m->Kpad, ep, m->d_status, s, m->nsm));
+    prof_close(m, ps_, s); }
+    ++launches;
+  }
+  { const int ps_ = prof_open(m, VIT_K_PREFIX, s);
+  prefix_tokens_kernel<<<dim3(m->nt, 1 + R, B), 32, 0, s>>>(m->cls, m->reg, m->pos, c.pos_on_cls, T, D, m->bn_res,
+                                                             S.x, S.xb, S.stats);
+  prof_close(m, ps_, s); }
+  CKL();
+  ++launches;
+
+  int tap_i = 0;
+  for (int l = 0; l < c.depth; ++l) {
+    const BlockW& bw = m->blocks[l];
+    // LN1 (folded) + QKV
+    {
+      const int bn = pick_bn(M, 3 * D, m->nsm);
+      EpiParams ep{};
+      ep.M = M;
+      ep.N = 3 * D;
+      ep.bias = bw.qkv_b;
+      ep.colsum = bw.qkv_c;
+      ep.stats_in = S.stats;
+      ep.nt = m->nt;
+      ep.nt_cols = m->bn_res;
+      ep.D = D;
+      ep.eps = c.ln_eps;
+      ep.out = S.big;
+      ep.ldo = 3 * D;
+      { const int ps_ = prof_open(m, VIT_K_QKV_GEMM, s);
+      CK(launch_gemm(bn, EPI_LNFOLD, tm_xb, bw.tm_qkv[bn == 256], M, 3 * D, D, ep, m->d_status, s, m->nsm));
+      prof_close(m, ps_, s); }
+      ++launches;
+    }
+    { const int ps_ = prof_open(m, VIT_K_ATTENTION, s);
+    CK(launch_attention(tm_qkv3, B, T, c.heads, S.attn, m->d_status, s));
+    prof_close(m, ps_, s); }
+    ++launches;
+    // proj + layer scale + residual
+    {
+      EpiParams ep{};
+      ep.M = M;
+      ep.N = D;
+      ep.bias = bw.proj_b;
+      ep.ls = bw.ls1;
+      ep.x = S.x;
+      ep.xb = S.xb;
+      ep.stats_out = S.stats;
+      { const int ps_ = prof_open(m, VIT_K_PROJ_GEMM, s);
+      CK(launch_gemm(m->bn_res, EPI_RESID, tm_attn, bw.tm_proj, M, D, D, ep, m->d_status, s, m->nsm));
+      prof_close(m, ps_, s); }
+      ++launches;
+    }
+    // LN2 (folded) + FC1 + GELU
+    {
+      const int bn = pick_bn(M, F, m->nsm);
+      EpiParams ep{};
+      ep.M = M;
+      ep.N = F;
+      ep.bias = bw.fc1_b;
+      ep.colsum = bw.fc1_c;
+      ep.stats_in = S.stats;
+      ep.nt = m->nt;
+      ep.nt_cols = m->bn_res;
+      ep.D = D;
+      ep.eps = c.ln_eps;
+      ep.out = S.big;
+      ep.ldo = F;
+      ep.gelu = 1;
+      { const int ps_ = prof_open(m, VIT_K_FC1_GEMM, s);
+      CK(launch_gemm(bn, EPI_LNFOLD, tm_xb, bw.tm_fc1[bn == 256], M, F, D, ep, m->d_status, s, m->nsm));
+      prof_close(m, ps_, s); }
+      ++launches;
+    }
+    // FC2 + layer scale + residual
+    {
+      EpiParams ep{};
+      ep.M = M;
+      ep.N = D;
+      ep.bias = bw.fc2_b;
+      ep.ls = bw.ls2;
+      ep.x = S.x;
+      ep.xb = S.xb;
+      ep.stats_out = S.stats;
+      { const int ps_ = prof_open(m, VIT_K_FC2_GEMM, s);
+      CK(launch_gemm(m->bn_res, EPI_RESID, tm_h, bw.tm_fc2, M, D, F, ep, m->d_status, s, m->nsm));
+      prof_close(m, ps_, s); }
+      ++launches;
+    }
+    if (out && out->hidden)
+      CK(cudaMemcpyAsync(out->hidden + static_cast<size_t>(l) * M * D, S.x, static_cast<size_t>(M) * D * 4,
+                         cudaMemcpyDeviceToDevice, s));
+    if (c.tap_mask & (1u << l)) {
+      if (out && out->taps[tap_i]) {
+        { const int ps_ = prof_open(m, VIT_K_TAP, s);
+        tap_kernel<<<dim3((P + 31) / 32, B), 256, 0, s>>>(S.x, m->norm_w, m->norm_b, T, R, D, c.ln_eps,
+                                                            out->taps[tap_i]);
+        prof_close(m, ps_, s); }
+        CKL();
+        ++launches;
+      }
+      ++tap_i;
+    }
+  }
+  if (out && (out->desc || out->patch_tokens)) {
+    const long long jobs = static_cast<long long>(B) * (1 + P);
+    { const int ps_ = prof_open(m, VIT_K_FINAL_LN, s);
+    final_ln_kernel<<<static_cast<int>((jobs + 7) / 8), 256, 0, s>>>(S.x, m->norm_w, m->norm_b, B, T, R, D, c.ln_eps,
+                                                                    out->desc, out->patch_tokens, out->patch_fp32);
+    prof_close(m, ps_, s); }
+    CKL();
+    ++launches;
+  }
+  m->last_launches = launches;
+  return VIT_OK;
+}
+
+vit_status check_outputs(const vit_outputs* out) {
+  if (!out) return VIT_OK;
+  if (!aligned16(out->desc) || !aligned16(out->patch_tokens) || !aligned16(out->hidden)) {
+    set_err("output pointers must be 16-byte aligned");
+    return VIT_E_INVALID_ARG;
+  }
+  for (int i = 0; i < 4; ++i)
+    if (!aligned16(out->taps[i])) {
+      set_err("tap pointers must be 16-byte aligned");
+      return VIT_E_INVALID_ARG;
+    }
+  return VIT_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ C ABI
+extern "C" {
+
+const char* vit_status_str(vit_status s) {
+  switch (s) {
+    case VIT_OK: return "ok";
+    case VIT_E_INVALID_ARG: return "invalid argument";
+    case VIT_E_SHAPE: return "shape mismatch";
+    case VIT_E_UNSUPPORTED: return "unsupported configuration";
+    case VIT_E_WORKSPACE: return "workspace too small";
+    case VIT_E_CUDA: return "CUDA error";
+    case VIT_E_DEVICE_TIMEOUT: return "device pipeline wait timed out";
+    case VIT_E_NONFINITE: return "non-finite value";
+  }
+  return "unknown status";
+}
+
+const char* vit_last_error(void) { return g_err.c_str(); }
+
+vit_status vit_create(const vit_config* cfg, const vit_weights* w, vit_model** out) {
+  if (!out) {
+    set_err("out is NULL");
+    return VIT_E_INVALID_ARG;
+  }
+  *out = nullptr;
+  vit_status st = validate_cfg(cfg);
+  if (st != VIT_OK) return st;
+  if (!w || !w->patch_w || !w->patch_b || !w->cls || !w->pos || !w->norm_w || !w->norm_b || !w->blocks ||
+      (cfg->n_registers > 0 && !w->reg)) {
+    set_err("missing weight pointer");
+    return VIT_E_INVALID_ARG;
+  }
+  for (int l = 0; l < cfg->depth; ++l) {
+    const vit_block_weights& b = w->blocks[l];
+    const void* ptrs[] = {b.ln1_w, b.ln1_b, b.qkv_w, b.qkv_b, b.proj_w, b.proj_b, b.ls1,
+                          b.ln2_w, b.ln2_b, b.fc1_w, b.fc1_b, b.fc2_w, b.fc2_b, b.ls2};
+    for (const void* p : ptrs)
+      if (!p || !aligned16(p)) {
+        set_err("block %d: weight pointer NULL or not 16-byte aligned", l);
+        return VIT_E_INVALID_ARG;
+      }
+  }
+  vit_model* m = new vit_model();
+  m->cfg = *cfg;
+  CK(cudaGetDevice(&m->device));
+  m->nsm = device_sms(m->device);
+  const int D = cfg->dim, F = cfg->mlp_dim, p = cfg->patch;
+  m->gh = cfg->img_h / p;
+  m->gw = cfg->img_w / p;
+  m->P = m->gh * m->gw;
+  m->T = 1 + cfg->n_registers + m->P;
+  m->K_pe = 3 * p * p;
+  m->Kpad = static_cast<int>(align_up(m->K_pe, 64));
+  m->bn_res = (D % 256 == 0) ? 256 : 128;
+  m->nt = D / m->bn_res;
+
+  cudaStream_t s;
+  auto fail = [&](vit_status e) {
+    vit_destroy(m);
+    return e;
+  };
+  if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) {
+    set_err("cudaStreamCreate failed");
+    return fail(VIT_E_CUDA);
+  }
+  auto run = [&]() -> vit_status {
+    vit_status e;
+    if ((e = alloc_dev(m, reinterpret_cast<void**>(&m->d_status), 16)) != VIT_OK) return e;
+    CK(cudaMemsetAsync(m->d_status, 0, 16, s));
+    if ((e = alloc_dev(m, reinterpret_cast<void**>(&m->patch_w), static_cast<size_t>(D) * m->Kpad * 2)) != VIT_OK)
+      return e;
+    pad_rows_bf16_kernel<<<grid_1d(static_cast<long long>(D) * m->Kpad, 256, m->nsm), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(w->patch_w), D, m->K_pe, m->Kpad, m->patch_w);
+    CKL();
+    const size_t npos = static_cast<size_t>(m->P + (cfg->pos_on_cls ? 1 : 0)) * D;
+    if ((e = to_f32(m, w->patch_b, D, &m->patch_b, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->pos, npos, &m->pos, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->cls, D, &m->cls, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->reg, static_cast<size_t>(cfg->n_registers) * D, &m->reg, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->norm_w, D, &m->norm_w, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->norm_b, D, &m->norm_b, s)) != VIT_OK) return e;
+    if (!tmap_2d(&m->tm_patch, m->patch_w, m->Kpad, D, m->Kpad, 64, m->bn_res)) return VIT_E_CUDA;
+    m->blocks.resize(cfg->depth);
+    for (int l = 0; l < cfg->depth; ++l) {
+      const vit_block_weights& src = w->blocks[l];
+      BlockW& b = m->blocks[l];
+      if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.qkv_wg), static_cast<size_t>(3) * D * D * 2)) != VIT_OK) return e;
+      if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.qkv_c), static_cast<size_t>(3) * D * 4)) != VIT_OK) return e;
+      if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.qkv_b), static_cast<size_t>(3) * D * 4)) != VIT_OK) return e;
+      if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.fc1_wg), static_cast<size_t>(F) * D * 2)) != VIT_OK) return e;
+      if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.fc1_c), static_cast<size_t>(F) * 4)) != VIT_OK) return e;
+      if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.fc1_b), static_cast<size_t>(F) * 4)) != VIT_OK) return e;
+      fold_ln_weight_kernel<<<3 * D, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(src.qkv_w), static_cast<const __nv_bfloat16*>(src.qkv_b),
+          static_cast<const __nv_bfloat16*>(src.ln1_w), static_cast<const __nv_bfloat16*>(src.ln1_b), 3 * D, D, b.qkv_wg,
+          b.qkv_c, b.qkv_b);
+      CKL();
+      fold_ln_weight_kernel<<<F, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(src.fc1_w), static_cast<const __nv_bfloat16*>(src.fc1_b),
+          static_cast<const __nv_bfloat16*>(src.ln2_w), static_cast<const __nv_bfloat16*>(src.ln2_b), F, D, b.fc1_wg,
+          b.fc1_c, b.fc1_b);
+      CKL();
+      b.proj_w = static_cast<const __nv_bfloat16*>(src.proj_w);
+      b.fc2_w = static_cast<const __nv_bfloat16*>(src.fc2_w);
+      if ((e = to_f32(m, src.proj_b, D, &b.proj_b, s)) != VIT_OK) return e;
+      if ((e = to_f32(m, src.ls1, D, &b.ls1, s)) != VIT_OK) return e;
+      if ((e = to_f32(m, src.fc2_b, D, &b.fc2_b, s)) != VIT_OK) return e;
+      if ((e = to_f32(m, src.ls2, D, &b.ls2, s)) != VIT_OK) return e;
+      if (!tmap_2d(&b.tm_qkv[0], b.qkv_wg, D, 3 * D, D, 64, 128) || !tmap_2d(&b.tm_fc1[0], b.fc1_wg, D, F, D, 64, 128) ||
+          !tmap_2d(&b.tm_proj, b.proj_w, D, D, D, 64, m->bn_res) ||
+          !tmap_2d(&b.tm_fc2, b.fc2_w, F, D, F, 64, m->bn_res))
+        return VIT_E_CUDA;
+      b.tm_qkv[1] = b.tm_qkv[0];
+      b.tm_fc1[1] = b.tm_fc1[0];
+      if ((3 * D) % 256 == 0 && !tmap_2d(&b.tm_qkv[1], b.qkv_wg, D, 3 * D, D, 64, 256)) return VIT_E_CUDA;
+      if (F % 256 == 0 && !tmap_2d(&b.tm_fc1[1], b.fc1_wg, D, F, D, 64, 256)) return VIT_E_CUDA;
+    }
+    CK(cudaStreamSynchronize(s));
+    return VIT_OK;
+  };
+  st = run();
+  cudaStreamDestroy(s);
+  if (st != VIT_OK) return fail(st);
+  *out = m;
+  return VIT_OK;
+}
+
+void vit_destroy(vit_model* m) {
+  if (!m) return;
+  for (cudaEvent_t e : m->prof_ev) cudaEventDestroy(e);
+  for (void* p : m->allocs) cudaFree(p);
+  delete m;
+}
+
+vit_status vit_workspace_size(const vit_model* m, int32_t batch, size_t* bytes) {
+  if (!m || !bytes) {
+    set_err("NULL argument");
+    return VIT_E_INVALID_ARG;
+  }
+  if (batch < 1 || batch > m->cfg.max_batch) {
+    set_err("batch %d outside 1..max_batch (%d)", batch, m->cfg.max_batch);
+    return VIT_E_SHAPE;
+  }
+  *bytes = ws_layout(m, batch).total;
+  return VIT_OK;
+}
+
+vit_status vit_forward(vit_model* m, const float* images, int32_t B, const vit_outputs* out, void* ws, size_t ws_bytes,
+                       vit_stream_t stream) {
+  if (!m || !images || !aligned16(images)) {
+    set_err("model or images NULL / images not 16-byte aligned");
+    return VIT_E_INVALID_ARG;
+  }
+  if (B < 1 || B > m->cfg.max_batch) {
+    set_err("batch %d outside 1..max_batch (%d)", B, m->cfg.max_batch);
+    return VIT_E_SHAPE;
+  }
+  vit_status st = check_outputs(out);
+  if (st != VIT_OK) return st;
+  const vit_config& c = m->cfg;
+  ImgSrc src{images, 3LL * c.img_h * c.img_w, static_cast<long long>(c.img_h) * c.img_w, c.img_w, 1, 0, 0, 0};
+  return run_forward(m, src, B, out, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+vit_status vit_host_workspace_size(const vit_model* m, int32_t batch, size_t* bytes) {
+  size_t fw = 0;
+  vit_status st = vit_workspace_size(m, batch, &fw);
+  if (st != VIT_OK) return st;
+  const size_t img = align_up(static_cast<size_t>(batch) * 3 * m->cfg.img_h * m->cfg.img_w * 4, 1024);
+  const size_t desc = align_up(static_cast<size_t>(batch) * m->cfg.dim * 4, 1024);
+  const size_t patch = align_up(static_cast<size_t>(batch) * m->P * m->cfg.dim * 2, 1024);
+  *bytes = img + desc + patch + fw;
+  return VIT_OK;
+}
+
+vit_status vit_forward_host(vit_model* m, const float* images_host, int32_t B, float* desc_host,
+                            void* patch_tokens_host, void* ws, size_t ws_bytes, vit_stream_t stream) {
+  if (!m || !images_host || !desc_host) {
+    set_err("model, images_host or desc_host is NULL");
+    return VIT_E_INVALID_ARG;
+  }
+  size_t need = 0;
+  vit_status st = vit_host_workspace_size(m, B, &need);
+  if (st != VIT_OK) return st;
+  if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) {
+    set_err("host-path workspace must be >= %zu bytes and 256-byte aligned", need);
+    return VIT_E_WORKSPACE;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t img_b = static_cast<size_t>(B) * 3 * m->cfg.img_h * m->cfg.img_w * 4;
+  const size_t img = align_up(img_b, 1024);
+  const size_t desc_b = static_cast<size_t>(B) * m->cfg.dim * 4;
+  const size_t desc = align_up(desc_b, 1024);
+  const size_t patch_b = static_cast<size_t>(B) * m->P * m->cfg.dim * 2;
+  const size_t patch = align_up(patch_b, 1024);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  float* d_img = reinterpret_cast<float*>(w8);
+  float* d_desc = reinterpret_cast<float*>(w8 + img);
+  void* d_patch = w8 + img + desc;
+  CK(cudaMemcpyAsync(d_img, images_host, img_b, cudaMemcpyHostToDevice, s));
+  vit_outputs o{};
+  o.desc = d_desc;
+  o.patch_tokens = patch_tokens_host ? d_patch : nullptr;
+  o.patch_fp32 = 0;
+  st = vit_forward(m, d_img, B, &o, w8 + img + desc + patch, ws_bytes - (img + desc + patch), stream);
+  if (st != VIT_OK) return st;
+  CK(cudaMemcpyAsync(desc_host, d_desc, desc_b, cudaMemcpyDeviceToHost, s));
+  if (patch_tokens_host) CK(cudaMemcpyAsync(patch_tokens_host, d_patch, patch_b, cudaMemcpyDeviceToHost, s));
+  return VIT_OK;
+}
+
+static int slide_count(int size, int side, int stride) {
+  if (size <= side) return 1;
+  return (size - side + stride - 1) / stride + 1;
+}
+
+vit_status vit_seg_workspace_size(const vit_model* m, int32_t H, int32_t W, int32_t C, int32_t mode, int32_t side,
+                                  int32_t stride, size_t* bytes) {
+  if (!m || !bytes || C < 1) {
+    set_err("NULL argument or C < 1");
+    return VIT_E_INVALID_ARG;
+  }
+  int nwin = 1;
+  if (mode == VIT_SEG_SLIDE) {
+    if (stride < 1 || side < 1) {
+      set_err("side and stride must be positive");
+      return VIT_E_INVALID_ARG;
+    }
+    nwin = slide_count(H, side, stride) * slide_count(W, side, stride);
+  }
+  size_t fw = 0;
+  vit_status st = vit_workspace_size(m, nwin, &fw);
+  if (st != VIT_OK) return st;
+  const size_t rows = static_cast<size_t>(nwin) * m->P;
+  *bytes = align_up(rows * m->cfg.dim * 4, 1024) + align_up(rows * 4, 1024) + align_up(rows * C * 4, 1024) + fw;
+  return VIT_OK;
+}
+
+vit_status vit_seg_zero_shot(vit_model* m, const float* image, int32_t H, int32_t W, const float* text, int32_t C,
+                             int32_t mode, int32_t side, int32_t stride, float* probs, int32_t* labels, void* ws,
+                             size_t ws_bytes, vit_stream_t stream) {
+  if (!m || !image || !text || !aligned16(image) || !aligned16(text) || !aligned16(probs) || !aligned16(labels)) {
+    set_err("NULL or misaligned pointer");
+    return VIT_E_INVALID_ARG;
+  }
+  const vit_config& c = m->cfg;
+  int ny = 1, nx = 1, g = 0;
+  if (mode == VIT_SEG_SLIDE) {
+    if (side != c.img_h || side != c.img_w || H < side || W < side) {
+      set_err("slide: side (%d) must equal the model input %dx%d and fit in the image %dx%d", side, c.img_h, c.img_w, H,
+              W);
+      return VIT_E_SHAPE;
+    }
+    ny = slide_count(H, side, stride);
+    nx = slide_count(W, side, stride);
+    g = m->gh;
+  } else if (mode == VIT_SEG_WHOLE) {
+    if (H != c.img_h || W != c.img_w) {
+      set_err("whole: image %dx%d must equal the model input %dx%d (no position-embedding resize)", H, W, c.img_h,
+              c.img_w);
+      return VIT_E_UNSUPPORTED;
+    }
+  } else {
+    set_err("mode must be VIT_SEG_WHOLE or VIT_SEG_SLIDE");
+    return VIT_E_INVALID_ARG;
+  }
+  size_t need = 0;
+  vit_status st = vit_seg_workspace_size(m, H, W, C, mode, side, stride, &need);
+  if (st != VIT_OK) return st;
+  if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) {
+    set_err("seg workspace must be >= %zu bytes and 256-byte aligned", need);
+    return VIT_E_WORKSPACE;
+  }
+  const int nwin = ny * nx;
+  const size_t rows = static_cast<size_t>(nwin) * m->P;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  float* tok = reinterpret_cast<float*>(w8);
+  size_t off = align_up(rows * c.dim * 4, 1024);
+  float* inv = reinterpret_cast<float*>(w8 + off);
+  off += align_up(rows * 4, 1024);
+  float* cosm = reinterpret_cast<float*>(w8 + off);
+  off += align_up(rows * C * 4, 1024);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  ImgSrc src{image, 0, static_cast<long long>(H) * W, W, nx, (mode == VIT_SEG_SLIDE) ? stride : 0,
+             (mode == VIT_SEG_SLIDE) ? H - side : 0, (mode == VIT_SEG_SLIDE) ? W - side : 0};
+  vit_outputs o{};
+  o.patch_tokens = tok;
+  o.patch_fp32 = 1;
+  st = run_forward(m, src, nwin, &o, w8 + off, ws_bytes - off, s);
+  if (st != VIT_OK) return st;
+  int launches = m->last_launches;
+  { const int ps_ = prof_open(m, VIT_K_SEG_NORM, s);
+  token_inv_norm_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(tok, static_cast<long long>(rows), c.dim, inv);
+  prof_close(m, ps_, s); }
+  CKL();
+  dim3 cg(static_cast<unsigned>((rows + 63) / 64), static_cast<unsigned>((C + 63) / 64));
+  { const int ps_ = prof_open(m, VIT_K_SEG_COS, s);
+  cos_gemm_kernel<<<cg, 256, 0, s>>>(tok, inv, text, m->P, static_cast<long long>(rows), C, c.dim, cosm);
+  prof_close(m, ps_, s); }
+  CKL();
+  launches += 2;
+  const long long pix = static_cast<long long>(H) * W;
+  if (mode == VIT_SEG_SLIDE) {
+    { const int ps_ = prof_open(m, VIT_K_SEG_MAP, s);
+    seg_slide_kernel<<<static_cast<int>((pix + 127) / 128), 128, 0, s>>>(cosm, C, g, H, W, side, stride, ny, nx, probs,
+                                                                         labels);
+    prof_close(m, ps_, s); }
+  } else {
+    { const int ps_ = prof_open(m, VIT_K_SEG_MAP, s);
+    seg_whole_kernel<<<static_cast<int>((pix + 127) / 128), 128, 0, s>>>(cosm, C, m->gh, m->gw, H, W, probs, labels);
+    prof_close(m, ps_, s); }
+  }
+  CKL();
+  m->last_launches = launches + 1;
+  return VIT_OK;
+}
+
+vit_status vit_poll(vit_model* m, vit_stream_t stream) {
+  if (!m) {
+    set_err("model is NULL");
+    return VIT_E_INVALID_ARG;
+  }
+  CK(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  int v = 0;
+  CK(cudaMemcpy(&v, m->d_status, 4, cudaMemcpyDeviceToHost));
+  if (v != 0) {
+    CK(cudaMemset(m->d_status, 0, 4));
+    set_err("a kernel gave up on a pipeline wait (site 0x%x)", v);
+    return VIT_E_DEVICE_TIMEOUT;
+  }
+  return VIT_OK;
+}
+
+int32_t vit_last_launch_count(const vit_model* m) { return m ? m->last_launches : 0; }
+
+vit_status vit_profile_begin(vit_model* m, int32_t capacity) {
+  if (!m || capacity < 1) {
+    set_err("model is NULL or capacity < 1");
+    return VIT_E_INVALID_ARG;
+  }
+  const size_t need = static_cast<size_t>(capacity) * 2;
+  while (m->prof_ev.size() < need) {
+    cudaEvent_t e;
+    CK(cudaEventCreate(&e));
+    m->prof_ev.push_back(e);
+  }
+  m->prof_kind.assign(capacity, -1);
+  m->prof_used = 0;
+  m->prof_on = true;
+  return VIT_OK;
+}
+
+vit_status vit_profile_end(vit_model* m, float* total_ms, int32_t* launches) {
+  if (!m) {
+    set_err("model is NULL");
+    return VIT_E_INVALID_ARG;
+  }
+  float acc[VIT_K_COUNT] = {};
+  int32_t cnt[VIT_K_COUNT] = {};
+  for (int i = 0; i < m->prof_used; ++i) {
+    CK(cudaEventSynchronize(m->prof_ev[2 * i + 1]));
+    float ms = 0.f;
+    CK(cudaEventElapsedTime(&ms, m->prof_ev[2 * i], m->prof_ev[2 * i + 1]));
+    const int k = m->prof_kind[i];
+    if (k >= 0 && k < VIT_K_COUNT) {
+      acc[k] += ms;
+      cnt[k] += 1;
+    }
+  }
+  m->prof_on = false;
+  m->prof_used = 0;
+  if (total_ms) std::memcpy(total_ms, acc, sizeof(acc));
+  if (launches) std::memcpy(launches, cnt, sizeof(cnt));
+  return VIT_OK;
+}
+
+// ------------------------------------------------------------------ stage entry points
+vit_status vit_stage_linear(const void* A, const void* W, const float* bias, int32_t M, int32_t N, int32_t K,
+                            int32_t gelu, void* out, int32_t* status, vit_stream_t stream) {
+  if (!A || !W || !bias || !out || !status || !aligned16(A) || !aligned16(W) || !aligned16(bias) || !aligned16(out)) {
+    set_err("NULL or misaligned pointer");
+    return VIT_E_INVALID_ARG;
+  }
+  if (M < 1 || N < 128 || N % 128 || K < 64 || K % 64) {
+    set_err("need M >= 1, N multiple of 128, K multiple of 64 (got %d, %d, %d)", M, N, K);
+    return VIT_E_SHAPE;
+  }
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  const int nsm = device_sms(dev);
+  const int bn = pick_bn(M, N, nsm);
+  CUtensorMap ta, tb;
+  if (!tmap_2d(&ta, A, K, M, K, 64, GEMM_BM) || !tmap_2d(&tb, W, K, N, K, 64, bn)) return VIT_E_CUDA;
+  EpiParams ep{};
+  ep.M = M;
+  ep.N = N;
+  ep.bias = bias;
+  ep.gelu = gelu;
+  ep.out = static_cast<__nv_bfloat16*>(out);
+  ep.ldo = N;
+  CK(launch_gemm(bn, EPI_BIAS, ta, tb, M, N, K, ep, status, reinterpret_cast<cudaStream_t>(stream), nsm));
+  return VIT_OK;
+}
+
+vit_status vit_stage_attention(const void* qkv, int32_t B, int32_t T, int32_t heads, void* out, int32_t* status,
+                               vit_stream_t stream) {
+  if (!qkv || !out || !status || !aligned16(qkv) || !aligned16(out)) {
+    set_err("NULL or misaligned pointer");
+    return VIT_E_INVALID_ARG;
+  }
+  if (B < 1 || T < 1 || heads < 1) {
+    set_err("need B, T, heads >= 1");
+    return VIT_E_SHAPE;
+  }
+  CUtensorMap tm;
+  if (!tmap_qkv3d(&tm, qkv, B, T, heads * 64)) return VIT_E_CUDA;
+  CK(launch_attention(tm, B, T, heads, static_cast<__nv_bfloat16*>(out), status,
+                      reinterpret_cast<cudaStream_t>(stream)));
+  return VIT_OK;
+}
+
+}  // extern "C"
