@@ -40,6 +40,26 @@ WORKLOAD_TEXT = {
 }
 
 
+def rank_image_seeds(wl, rank: int):
+    """Seeds of the two alternating input batches of one rank: every rank draws its own images
+    (weak scaling -- per-rank work is fixed and ranks never exchange data)."""
+    return [wl.image_seed + 1000 * rank + k for k in range(2)]
+
+
+def allreduce_max(x: float, dist, device) -> float:
+    """Max over ranks of a per-rank time (identity without a process group)."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def images_per_s(world: int, batch: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: all ranks' images over the slowest rank's time."""
+    return world * batch * steps / (ms_max / 1000.0)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -226,6 +246,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -250,7 +271,7 @@ def main(argv=None):
     weights = S.make_weights(spec, wl.weight_seed, wl.outlier)
     enc = V.VitEncoder(spec, weights, max_batch=B)
     # two input buffers alternate between steps (2 x 100 MB for ViT-L b8: more than the 126 MB L2)
-    imgs = [S.make_images(spec, B, wl.image_seed + 1000 * rank + k).cuda() for k in range(2)]
+    imgs = [S.make_images(spec, B, seed).cuda() for seed in rank_image_seeds(wl, rank)]
     outs = enc.alloc_outputs(B, desc=True, patch=True, patch_fp32=False)
     stream = torch.cuda.current_stream()
 
@@ -280,14 +301,32 @@ def main(argv=None):
     clk = clocks.stop()
     prof = enc.profile_end()
     enc.poll()
-    ms_total = e0.elapsed_time(e1)
-    t = torch.tensor([ms_total], dtype=torch.float64, device="cuda")
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
-    value = world * B * args.steps / (ms_total / 1000.0)
+    ms_total = allreduce_max(e0.elapsed_time(e1), dist, "cuda")
+    value = images_per_s(world, B, args.steps, ms_total)
 
     # ---- end to end through vit_forward_host: pinned host images in, descriptor + patch tokens out
+    e2e = None
+    if not args.no_e2e:
+        e2e = end_to_end(enc, imgs, spec, B, args, stream, barrier, dist, world)
+
+    peaks = load_peaks()
+    line = None
+    if rank == 0:
+        line = report(args, spec, wl, B, world, prof, ms_total, value, e2e, launches_per_step, clk, peaks, imgs, enc)
+    enc.close()
+    if rank == 0:
+        if not args.no_secondary:
+            line["secondary"] = [secondary_rate(V, "vits16_336_b64_outlier"), secondary_rate(V, "vits16_336_b1")]
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def end_to_end(enc, imgs, spec, B, args, stream, barrier, dist, world):
     host_imgs = [im.cpu().pin_memory() for im in imgs]
     desc_h = torch.empty(B, spec.dim, dtype=torch.float32).pin_memory()
     patch_h = torch.empty(B, spec.n_patches, spec.dim, dtype=torch.bfloat16).pin_memory()
@@ -304,73 +343,61 @@ def main(argv=None):
     torch.cuda.synchronize()
     barrier()
     enc.poll()
-    t2 = torch.tensor([f0.elapsed_time(f1)], dtype=torch.float64, device="cuda")
-    if dist is not None:
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-    e2e_value = world * B * args.steps / (float(t2.item()) / 1000.0)
+    e2e_value = images_per_s(world, B, args.steps, allreduce_max(f0.elapsed_time(f1), dist, "cuda"))
     h2d = host_imgs[0].numel() * 4
     d2h = desc_h.numel() * 4 + patch_h.numel() * 2
 
-    peaks = load_peaks()
-    line = None
-    if rank == 0:
-        flops = kernel_flops(spec, B)
-        nbytes = kernel_bytes(spec, B)
-        kernels = {}
-        for k, (ms, n) in prof.items():
-            entry = {"launches": n, "total_ms": ms, "avg_ms": ms / n, "share": ms / max(1e-9, sum(v[0] for v in prof.values()))}
-            if k in flops:
-                entry["tflops"] = flops[k] / (ms / n / 1000.0) / 1e12
-            if k in nbytes:
-                entry["gbs"] = nbytes[k] / (ms / n / 1000.0) / 1e9
-            kernels[k] = entry
-        top = max(prof, key=lambda k: prof[k][0])
-        avg_s = prof[top][0] / prof[top][1] / 1000.0
-        if top in flops:
-            ach = flops[top] / avg_s / 1e12
-            peak = peaks["bf16_tflops_sustained"]
-            roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-                    "traffic": None, "kernel": top, "flops_per_launch": flops[top],
-                    "peak_kind": f"bf16 dense, sustained ({peaks['source']})"}
-        else:
-            ach = nbytes.get(top, 0) / avg_s / 1e9
-            peak = peaks["hbm_gbs"]
-            roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                    "traffic": None, "kernel": top, "peak_kind": f"HBM copy ({peaks['source']})"}
-        step_flops = total_flops(spec, B)
-        line = {
-            "metric": METRIC, "value": value, "unit": "images/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD_TEXT[wl.name], "batch_per_gpu": B, "global_batch": B * world,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "two input buffers alternate (2 x %.0f MB); weights %.0f MB and activations per step "
-                             "exceed the 126 MB L2" % (imgs[0].numel() * 4 / 1e6, sum(
-                                 p.numel() * 2 for p in enc.w.values()) / 1e6 + sum(
-                                 p.numel() * 2 for b in enc.wb for p in b.values()) / 1e6),
-                       "timing": "CUDA events on the launching stream; per-launch events recorded inside the "
-                                 "timed region for the kernel breakdown"},
-            "tflops_per_gpu": step_flops / (ms_total / args.steps / 1000.0) / 1e12,
-            "frac_of_bf16_peak": {"measured_burst": step_flops / (ms_total / args.steps / 1000.0) / 1e12 /
-                                  peaks["bf16_tflops"], "spec_dense_2250": step_flops / (
-                                      ms_total / args.steps / 1000.0) / 1e12 / 2250.0},
-            "roofline": roof,
-            "kernels": kernels,
-            "e2e": {"value": e2e_value, "unit": "images/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk,
-        }
-    enc.close()
-    if rank == 0:
-        if not args.no_secondary:
-            line["secondary"] = [secondary_rate(V, "vits16_336_b64_outlier"), secondary_rate(V, "vits16_336_b1")]
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(wl)
-        print(json.dumps(line), flush=True)
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
-    return 0
+    return {"value": e2e_value, "unit": "images/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def report(args, spec, wl, B, world, prof, ms_total, value, e2e, launches_per_step, clk, peaks, imgs, enc):
+    flops = kernel_flops(spec, B)
+    nbytes = kernel_bytes(spec, B)
+    kernels = {}
+    for k, (ms, n) in prof.items():
+        entry = {"launches": n, "total_ms": ms, "avg_ms": ms / n, "share": ms / max(1e-9, sum(v[0] for v in prof.values()))}
+        if k in flops:
+            entry["tflops"] = flops[k] / (ms / n / 1000.0) / 1e12
+        if k in nbytes:
+            entry["gbs"] = nbytes[k] / (ms / n / 1000.0) / 1e9
+        kernels[k] = entry
+    top = max(prof, key=lambda k: prof[k][0])
+    avg_s = prof[top][0] / prof[top][1] / 1000.0
+    if top in flops:
+        ach = flops[top] / avg_s / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                "traffic": None, "kernel": top, "flops_per_launch": flops[top],
+                "peak_kind": f"bf16 dense, sustained ({peaks['source']})"}
+    else:
+        ach = nbytes.get(top, 0) / avg_s / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                "traffic": None, "kernel": top, "peak_kind": f"HBM copy ({peaks['source']})"}
+    step_flops = total_flops(spec, B)
+    line = {
+        "metric": METRIC, "value": value, "unit": "images/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[wl.name], "batch_per_gpu": B, "global_batch": B * world,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "two input buffers alternate (2 x %.0f MB); weights %.0f MB and activations per step "
+                         "exceed the 126 MB L2" % (imgs[0].numel() * 4 / 1e6, sum(
+                             p.numel() * 2 for p in enc.w.values()) / 1e6 + sum(
+                             p.numel() * 2 for b in enc.wb for p in b.values()) / 1e6),
+                   "timing": "CUDA events on the launching stream; per-launch events recorded inside the "
+                             "timed region for the kernel breakdown"},
+        "tflops_per_gpu": step_flops / (ms_total / args.steps / 1000.0) / 1e12,
+        "frac_of_bf16_peak": {"measured_burst": step_flops / (ms_total / args.steps / 1000.0) / 1e12 /
+                              peaks["bf16_tflops"], "spec_dense_2250": step_flops / (
+                                  ms_total / args.steps / 1000.0) / 1e12 / 2250.0},
+        "roofline": roof,
+        "kernels": kernels,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    return line
 
 
 if __name__ == "__main__":

@@ -27,7 +27,9 @@ def desc_cos(g, r):
     return float((g * r).sum() / (np.linalg.norm(g) * np.linalg.norm(r)))
 
 
-def run_gpu(spec, weights, images, hidden=True, patch=True, taps=None):
+def run_gpu(spec, weights, images, hidden=True, patch=True, taps=None, keep=None):
+    """Run vit_forward on the whole batch; ``keep`` (image indices) limits what is copied back
+    of the per-block hidden states (the rest of the outputs come back whole)."""
     import vision_transformer_encoder_fwd_b200 as V
     B = images.shape[0]
     enc = V.VitEncoder(spec, weights, max_batch=B)
@@ -37,6 +39,12 @@ def run_gpu(spec, weights, images, hidden=True, patch=True, taps=None):
     enc.poll()
     res = {}
     for k, v in outs.items():
+        if k == "hidden" and keep is not None:
+            res[k] = np.zeros((v.shape[0], v.shape[1]) + tuple(v.shape[2:]), dtype=np.float32)
+            res["hidden_finite"] = bool(torch.isfinite(v).all().item())
+            for i in keep:
+                res[k][:, i] = v[:, i].cpu().numpy()
+            continue
         res[k] = [t.double().cpu().numpy() for t in v] if isinstance(v, list) else v.double().cpu().numpy()
     res["launches"] = enc.last_launch_count()
     enc.close()

@@ -2,23 +2,33 @@
 //
 // "DINOv2 n semantic" diagram, panel "Encoder self-attention": per head, softmax over keys of
 // Q K^T / sqrt(64), times V, heads merged.  kornia/dinov3 card, "Build BF16, not FP16": the
-// scaled logits reach ~2.5e6, so Q, K, V and P stay bf16 but the logits, the running maximum
+// scaled logits reach ~2.5e6, so Q, K, V and P stay bf16 while the logits, the running maximum
 // and the running sum are fp32 (fp32's exponent range).
 //
-// One CTA per (128-query tile, head, image); 6 warps:
-//   warp 0 (one lane)  TMA: the Q tile once, then K_j and V_j (128 keys x 64 dims each) into a
-//                      2-deep ring, read straight from the stacked QKV activation [B, T, 3D]
-//                      through a 3-D tensor map (rows past T are zero-filled).
-//   warp 1             allocates 256 TMEM columns; one lane issues S = Q K_j^T (M=128, N=128)
-//                      into TMEM columns 0..127 and O_j = P_j V_j (M=128, N=64, V as an
-//                      MN-major operand) into columns 128 + 64 (j % 2).
-//   warps 2..5         softmax, one query row per thread (TMEM lane = row): row maximum over
-//                      the valid keys, exp2 of (s - max) * log2(e) / 8, P_j written to shared
-//                      memory in the 128-byte-swizzled K-major layout the MMA reads, running
-//                      sum; the fp32 output row is kept in registers and rescaled as
-//                      O <- alpha O + P_j V_j when each P_j V_j lands.
-// Two CTAs fit on one SM (112 KB shared memory and 256 TMEM columns each), so one CTA's
-// softmax overlaps the other's MMAs.
+// One CTA per (pair of 128-query tiles, head, image); 10 warps, one CTA per SM:
+//   warp 0 (one lane)  TMA: K_j and V_j (128 keys x 64 dims each) into a 3-deep ring, read from
+//                      the stacked QKV activation [B, T, 3D] through a 3-D tensor map (rows past
+//                      T are zero-filled).
+//   warp 1             allocates all 512 TMEM columns; one lane issues, per key block j and
+//                      query tile i:  O_i += P_i [V_j | 1]  (A = P_i from TMEM; B = V_j, MN-major,
+//                      extended by a constant column of ones, N = 80), then S_i = Q_i K_{j+1}^T
+//                      with Q_i also read from TMEM, so shared memory only feeds K and V.
+//                      The tensor pipe executes one thread's MMAs in issue order, so S_i may
+//                      overwrite the columns that held P_i.  Column 64 of O_i accumulates
+//                      sum_k P_ik in fp32 -- the softmax denominator of exactly the bf16 P that
+//                      multiplies V.
+//   warps 2..5, 6..9   softmax of query tile 0 and 1, one query row per thread (TMEM lane =
+//                      row).  First each thread copies its Q row from global memory into TMEM.
+//                      Per key block: one 128-column load of S_i, row maximum over the valid
+//                      keys, P = 2^((s - m) log2(e) / 8) -- exponent pairs from one packed fp32
+//                      FMA, the exponential from the special-function unit for most keys and from
+//                      a cubic on the FMA pipe for the rest -- packed to bf16 and written into the
+//                      first 64 columns of S_i.  The running maximum is only moved when it grows
+//                      by more than 2^8 (O_i, including its sum column, is then rescaled in TMEM
+//                      first), so every P stays <= 256.
+// TMEM: S_0 [0,128), S_1 [128,256), O_0 [256,336), O_1 [336,416), Q_0 [416,448), Q_1 [448,480)
+// (32-bit columns, lane = row; Q and P hold two bf16 per column).
+// While one softmax group works on S_0 the tensor pipe runs the other tile's MMAs.
 #pragma once
 
 #include "common.cuh"
@@ -27,69 +37,157 @@ namespace vit {
 
 constexpr int ATT_BM = 128;
 constexpr int ATT_BN = 128;
-constexpr int ATT_THREADS = 192;
+constexpr int ATT_THREADS = 320;
+constexpr int ATT_KV_STAGES = 3;
 
 struct AttnCfg {
-  static constexpr int Q_BYTES = ATT_BM * 64 * 2;  // 16 KB
-  static constexpr int K_BYTES = ATT_BN * 64 * 2;  // 16 KB
-  static constexpr int V_BYTES = ATT_BN * 64 * 2;  // 16 KB
-  static constexpr int P_BYTES = ATT_BM * ATT_BN * 2;  // 32 KB: two 64-key swizzle atoms
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + 2 * K_BYTES;
-  static constexpr int OFF_P = OFF_V + 2 * V_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
-  static constexpr int SMEM_BYTES = OFF_BAR + 128;
-  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr int K_BYTES = ATT_BN * 64 * 2;   // 16 KB
+  static constexpr int V_BYTES = ATT_BN * 64 * 2;   // 16 KB
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + ATT_KV_STAGES * K_BYTES;
+  // the constant "ones" MN-major atom that extends every V stage by 16 columns (1, 0, ..., 0)
+  static constexpr int OFF_ONES = OFF_V + ATT_KV_STAGES * V_BYTES;
+  static constexpr int OFF_BAR = OFF_ONES + V_BYTES;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256;
+  static_assert(8 * (2 * ATT_KV_STAGES + 8) + 8 <= 256, "barrier area too small");
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int O_COLS = 80;                 // 64 output columns + the sum column + padding
+  static constexpr uint32_t TM_S = 0, TM_O = 256, TM_Q = 416;
 };
 
 // log2(e) / sqrt(64)
 constexpr float kAttnScaleLog2 = 0.18033688011112042f;
+// The running maximum moves only when a row's maximum grows by more than 2^8.
+constexpr float kRescaleLog2 = 8.0f;
 
-__global__ void __launch_bounds__(ATT_THREADS, 2)
-    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, int T, int D, __nv_bfloat16* __restrict__ out,
-                       int* gstatus) {
+// Of every 8 keys, this many take the FMA-pipe exponential (the rest the special-function unit).
+constexpr int kPolyPer8 = 2;
+
+// 2^x on the FMA pipe for a pair of values: x = j + f with j = round(x) (add 1.5 * 2^23) and
+// |f| <= 1/2, 2^f from a cubic (Remez fit of the relative error, max 7.5e-5; see
+// gen_exp2_poly.py), 2^j added into the exponent field.  x is clamped at -125 so that the
+// result stays a normal float.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 j = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = fadd2(x, make_float2(-j.x, -j.y));
+  float2 p = ffma2(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.242611125f, 0.242611125f));
+  p = ffma2(p, f, make_float2(0.693260968f, 0.693260968f));
+  p = ffma2(p, f, make_float2(0.999928057f, 0.999928057f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Row maximum of 128 logits with four independent 3-input max chains.
+__device__ __forceinline__ float row_max128(const float (&s)[128]) {
+  float m0 = fmaxf(s[0], s[1]), m1 = fmaxf(s[2], s[3]), m2 = fmaxf(s[4], s[5]), m3 = fmaxf(s[6], s[7]);
+#pragma unroll
+  for (int t = 8; t < 128; t += 8) {
+    m0 = fmax3(m0, s[t], s[t + 1]);
+    m1 = fmax3(m1, s[t + 2], s[t + 3]);
+    m2 = fmax3(m2, s[t + 4], s[t + 5]);
+    m3 = fmax3(m3, s[t + 6], s[t + 7]);
+  }
+  return fmax3(m0, m1, fmaxf(m2, m3));
+}
+
+// P for one row of one key block: p = 2^(s * c - m * c) for pairs of keys (one packed fp32 FMA
+// forms the exponent pair); masked keys carry s = -inf and come out as 0 (the FMA-pipe path
+// clamps them to 2^-125 and they are zeroed explicitly).  Each 32-key chunk is packed to bf16
+// and stored to TMEM (16 columns from t_p) as soon as it is done; one wait covers the stores.
+template <bool MASK>
+__device__ __forceinline__ void softmax_block_p(const float (&s)[128], float mc, int valid, uint32_t t_p) {
+  const float2 cc = make_float2(kAttnScaleLog2, kAttnScaleLog2);
+  const float2 nm = make_float2(-mc, -mc);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int u = 0; u < 32; u += 2) {
+      const int t = c * 32 + u;
+      const float2 x = ffma2(make_float2(s[t], s[t + 1]), cc, nm);
+      float2 e;
+      if ((t & 7) >= 8 - kPolyPer8) {
+        e = exp2_fma2(x);
+        if (MASK) {
+          e.x = (t < valid) ? e.x : 0.f;
+          e.y = (t + 1 < valid) ? e.y : 0.f;
+        }
+      } else {
+        e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      }
+      pk[u >> 1] = pack_bf16x2(e.x, e.y);
+    }
+    tmem_st16_nowait(t_p + c * 16, pk);
+  }
+  tmem_st_wait();
+}
+
+__global__ void __launch_bounds__(ATT_THREADS, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __nv_bfloat16* __restrict__ qkv, int T, int D,
+                       __nv_bfloat16* __restrict__ out, int* gstatus) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  // The swizzled layouts assume 1024-byte aligned tiles; report and stop if the shared
-  // window is not (uniform across the CTA, before anything is allocated).
+  // The swizzled layouts assume 1024-byte aligned tiles; report and stop if the shared window
+  // is not (uniform across the CTA, before anything is allocated).
   if ((smem_u32(smem) & 1023u) != 0) {
     if (threadIdx.x == 0) atomicExch(gstatus, DEV_TIMEOUT_ATTN + 15);
     return;
   }
-  uint8_t* sQ = smem + AttnCfg::OFF_Q;
   uint8_t* sK = smem + AttnCfg::OFF_K;
   uint8_t* sV = smem + AttnCfg::OFF_V;
-  uint8_t* sP = smem + AttnCfg::OFF_P;
-  uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + AttnCfg::OFF_BAR);
-  uint64_t* kv_full = q_full + 1;    // [2]
-  uint64_t* kv_empty = q_full + 3;   // [2]
-  uint64_t* s_full = q_full + 5;
-  uint64_t* p_full = q_full + 6;
-  uint64_t* pv_full = q_full + 7;    // [2]
-  uint64_t* mma_done = q_full + 9;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(q_full + 10);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnCfg::OFF_BAR);
+  uint64_t* kv_full = bars;                               // [ATT_KV_STAGES]
+  uint64_t* kv_empty = kv_full + ATT_KV_STAGES;           // [ATT_KV_STAGES]
+  uint64_t* s_full = kv_empty + ATT_KV_STAGES;            // [2]
+  uint64_t* p_full = s_full + 2;                          // [2]
+  uint64_t* pv_done = p_full + 2;                         // [2]
+  uint64_t* mma_done = pv_done + 2;                       // 1
+  uint64_t* q_ready = mma_done + 1;                       // 1: both Q tiles copied into TMEM
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(q_ready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qblk = blockIdx.x;
+  const int n_qtiles = (T + ATT_BM - 1) / ATT_BM;
+  const int tile0 = blockIdx.x * 2;
+  const int ntile = min(2, n_qtiles - tile0);
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int nkv = (T + ATT_BN - 1) / ATT_BN;
 
   if (threadIdx.x == 0) {
     *abort_flag = (*reinterpret_cast<volatile int*>(gstatus) != 0) ? 1 : 0;
-    mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    mbar_init(q_ready, 128 * ntile);
+    for (int s = 0; s < ATT_KV_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
-      mbar_init(&pv_full[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&pv_done[i], 1);
+    }
     mbar_init(mma_done, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmQKV);
+  }
+  {
+    // The ones atom: 128 key rows of 128 bytes in the 128-byte-swizzled MN-major layout, value
+    // 1.0 at N position 0 of every row (16-byte chunk 0, swizzled to chunk r % 8), 0 elsewhere.
+    uint4* ones = reinterpret_cast<uint4*>(smem + AttnCfg::OFF_ONES);
+    for (int i = threadIdx.x; i < AttnCfg::V_BYTES / 16; i += blockDim.x) {
+      const int row = i >> 3, chunk = i & 7;
+      ones[i] = make_uint4((chunk == (row & 7)) ? 0x3F80u : 0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, AttnCfg::TMEM_COLS);
@@ -103,13 +201,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
 
   if (!skip && warp == 0 && lane == 0) {
     // ------------------------------------------------------------------ TMA producer
-    int issued_parity[3] = {-1, -1, -1};  // q_full, kv_full[0], kv_full[1]
-    mbar_arrive_expect_tx(q_full, AttnCfg::Q_BYTES);
-    tma_load_3d(sQ, &tmQKV, h * 64, qblk * ATT_BM, b, q_full);
-    issued_parity[0] = 0;
+    int issued_parity[1 + ATT_KV_STAGES];
+    for (int s = 0; s <= ATT_KV_STAGES; ++s) issued_parity[s] = -1;
     for (int j = 0; j < nkv; ++j) {
-      const int s = j & 1;
-      const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
+      const int s = j % ATT_KV_STAGES;
+      const uint32_t ph = static_cast<uint32_t>(j / ATT_KV_STAGES) & 1u;
       if (!mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 1)) break;
       mbar_arrive_expect_tx(&kv_full[s], AttnCfg::K_BYTES + AttnCfg::V_BYTES);
       tma_load_3d(sK + s * AttnCfg::K_BYTES, &tmQKV, D + h * 64, j * ATT_BN, b, &kv_full[s]);
@@ -117,154 +213,182 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       issued_parity[1 + s] = static_cast<int>(ph);
     }
     if (*abort_flag) {
-      if (issued_parity[0] >= 0) mbar_wait_drain(q_full, 0);
-      for (int s = 0; s < 2; ++s)
+      for (int s = 0; s < ATT_KV_STAGES; ++s)
         if (issued_parity[1 + s] >= 0) mbar_wait_drain(&kv_full[s], static_cast<uint32_t>(issued_parity[1 + s]));
     }
   } else if (!skip && warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(ATT_BM, ATT_BN, false);
-      constexpr uint32_t idesc_o = idesc_bf16(ATT_BM, 64, true);
-      const uint32_t q0 = smem_u32(sQ);
+      constexpr uint32_t idesc_o = idesc_bf16(ATT_BM, AttnCfg::O_COLS, true);
       const uint32_t k0 = smem_u32(sK);
       const uint32_t v0 = smem_u32(sV);
-      const uint32_t p0 = smem_u32(sP);
-      bool ok = mbar_wait(q_full, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 2) &&
+      const uint32_t ones0 = smem_u32(smem + AttnCfg::OFF_ONES);
+      // Every MMA operand is built once: K and V descriptors per stage and K step (a K step only
+      // moves the start address: +32 bytes for K, +2048 for V), TMEM addresses per tile.  Each
+      // chain of MMAs into one accumulator is then issued by a single asm statement.
+      // Stage st moves the K start address by st * K_BYTES and the V start address by
+      // st * V_BYTES while the V leading byte offset (distance to the ones atom) shrinks by the
+      // same amount: both are linear in st, so the stage descriptors are one add away.
+      uint64_t dk0[4], dv0[8];
+      {
+        const uint64_t d0 = sdesc_sw128(k0, 16, 1024);
+        const uint64_t v0d = sdesc_sw128(v0, ones0 - v0, 1024);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dk0[k] = d0 + 2 * k;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) dv0[kk] = v0d + 128 * kk;
+      }
+      constexpr uint64_t kStepK = AttnCfg::K_BYTES >> 4;
+      constexpr uint64_t kStepV = (AttnCfg::V_BYTES >> 4) - (static_cast<uint64_t>(AttnCfg::V_BYTES >> 4) << 16);
+      const uint32_t t_s0 = tmem_base + AttnCfg::TM_S, t_q0 = tmem_base + AttnCfg::TM_Q;
+      const uint32_t t_o0 = tmem_base + AttnCfg::TM_O;
+      uint32_t aq[2][4], ap[2][8];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) aq[i][k] = t_q0 + i * 32 + k * 8;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) ap[i][kk] = t_s0 + i * 128 + kk * 8;
+      }
+      bool ok = mbar_wait(q_ready, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 2) &&
                 mbar_wait(&kv_full[0], 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 3);
       if (ok) {
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          tc_mma_ss(tmem_base, sdesc_sw128(q0 + k * 32, 16, 1024), sdesc_sw128(k0 + k * 32, 16, 1024), idesc_s,
-                    k > 0 ? 1u : 0u);
-        tc_commit(s_full);
+        for (int i = 0; i < ntile; ++i) {
+          tc_mma_ts_chain4(t_s0 + i * 128, aq[i], dk0, idesc_s, 0u);
+          tc_commit(&s_full[i]);
+        }
       }
       for (int j = 0; ok && j < nkv; ++j) {
-        if (!mbar_wait(p_full, static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 4)) break;
-        tc_fence_after();
-        if (j + 1 < nkv) {
-          const int s1 = (j + 1) & 1;
-          if (!mbar_wait(&kv_full[s1], static_cast<uint32_t>((j + 1) >> 1) & 1u, abort_flag, gstatus,
-                         DEV_TIMEOUT_ATTN + 5))
+        const int s = j % ATT_KV_STAGES;
+        const int s1 = (j + 1) % ATT_KV_STAGES;
+        uint64_t dvs[8], dk1[4];
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) dvs[kk] = dv0[kk] + static_cast<uint64_t>(s) * kStepV;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dk1[k] = dk0[k] + static_cast<uint64_t>(s1) * kStepK;
+        for (int i = 0; i < ntile && ok; ++i) {
+          if (!mbar_wait(&p_full[i], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 4)) {
+            ok = false;
             break;
+          }
           tc_fence_after();
-          const uint32_t kb = k0 + s1 * AttnCfg::K_BYTES;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma_ss(tmem_base, sdesc_sw128(q0 + k * 32, 16, 1024), sdesc_sw128(kb + k * 32, 16, 1024), idesc_s,
-                      k > 0 ? 1u : 0u);
-          tc_commit(s_full);
+          tc_mma_ts_chain8(t_o0 + i * AttnCfg::O_COLS, ap[i], dvs, idesc_o, j > 0 ? 1u : 0u);
+          tc_commit(&pv_done[i]);
+          if (j + 1 < nkv) {
+            if (i == 0) {
+              if (!mbar_wait(&kv_full[s1], static_cast<uint32_t>((j + 1) / ATT_KV_STAGES) & 1u, abort_flag, gstatus,
+                             DEV_TIMEOUT_ATTN + 5)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            tc_mma_ts_chain4(t_s0 + i * 128, aq[i], dk1, idesc_s, 0u);
+            tc_commit(&s_full[i]);
+          }
         }
-        const int s = j & 1;
-        const uint32_t vb = v0 + s * AttnCfg::V_BYTES;
-        const uint32_t d_o = tmem_base + 128u + static_cast<uint32_t>(s * 64);
-#pragma unroll
-        for (int kk = 0; kk < ATT_BN / 16; ++kk) {
-          const uint32_t pa = p0 + (kk >> 2) * (AttnCfg::P_BYTES / 2) + (kk & 3) * 32;
-          tc_mma_ss(d_o, sdesc_sw128(pa, 16, 1024), sdesc_sw128(vb + kk * 2048, AttnCfg::V_BYTES, 1024), idesc_o,
-                    kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&pv_full[s]);
-        tc_commit(&kv_empty[s]);
+        if (ok) tc_commit(&kv_empty[s]);
       }
       tc_commit(mma_done);
     }
     __syncwarp();
   } else if (!skip && warp >= 2) {
-    // ------------------------------------------------------------------ softmax
-    const int q = warp & 3;
-    const int r = q * 32 + lane;
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    float o[64];
+    // ------------------------------------------------------------------ softmax groups
+    const int wg = (warp - 2) >> 2;
+    if (wg < ntile) {
+      const int q = warp & 3;
+      const int r = q * 32 + lane;
+      const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+      const uint32_t t_s = tmem_base + lane_off + AttnCfg::TM_S + wg * 128;
+      const uint32_t t_o = tmem_base + lane_off + AttnCfg::TM_O + wg * AttnCfg::O_COLS;
+      {
+        // this thread's query row (64 bf16 = 32 columns, two per column) into TMEM
+        const int qrow = (tile0 + wg) * ATT_BM + r;
+        uint32_t qv[32];
+        if (qrow < T) {
+          const uint4* src = reinterpret_cast<const uint4*>(qkv + (static_cast<size_t>(b) * T + qrow) * (3 * D) + h * 64);
 #pragma unroll
-    for (int i = 0; i < 64; ++i) o[i] = 0.f;
-    float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      if (!mbar_wait(s_full, static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 6)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const int valid = min(ATT_BN, T - j * ATT_BN);
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < ATT_BN / 32; ++c) {
-        float v[32];
-        __syncwarp();
-        tmem_ld32(lane_base + c * 32, v);
+          for (int t = 0; t < 8; ++t) {
+            const uint4 w = __ldg(src + t);
+            qv[4 * t] = w.x;
+            qv[4 * t + 1] = w.y;
+            qv[4 * t + 2] = w.z;
+            qv[4 * t + 3] = w.w;
+          }
+        } else {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const float sv = (c * 32 + t < valid) ? v[t] : -INFINITY;
-          mx = fmaxf(mx, sv);
+          for (int t = 0; t < 32; ++t) qv[t] = 0u;
         }
+        __syncwarp();
+        tmem_st32(tmem_base + lane_off + AttnCfg::TM_Q + wg * 32, qv);
+        tc_fence_before();
+        mbar_arrive(q_ready);
       }
-      const float m_new = fmaxf(m, mx);
-      const float alpha = ex2_approx((m - m_new) * kAttnScaleLog2);
-      const float mc = m_new * kAttnScaleLog2;
-      if (j > 0) {
-        const int s = (j - 1) & 1;
-        if (!mbar_wait(&pv_full[s], static_cast<uint32_t>((j - 1) >> 1) & 1u, abort_flag, gstatus,
-                       DEV_TIMEOUT_ATTN + 7)) {
+      float m = -INFINITY;
+      bool ok = true;
+      for (int j = 0; j < nkv; ++j) {
+        if (!mbar_wait(&s_full[wg], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 6)) {
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float v[32];
-          __syncwarp();
-          tmem_ld32(lane_base + 128u + static_cast<uint32_t>(s * 64 + c * 32), v);
-#pragma unroll
-          for (int t = 0; t < 32; ++t) o[c * 32 + t] = fmaf(o[c * 32 + t], alpha_prev, v[t]);
-        }
-      }
-      float rs = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < ATT_BN / 32; ++c) {
-        float v[32];
+        float s[128];
         __syncwarp();
-        tmem_ld32(lane_base + c * 32, v);
-        uint32_t pk[16];
+        tmem_ld128(t_s, s);
+        const int valid = min(ATT_BN, T - j * ATT_BN);
+        if (valid < ATT_BN) {
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const int k0 = c * 32 + 2 * t;
-          const float e0 = (k0 < valid) ? ex2_approx(fmaf(v[2 * t], kAttnScaleLog2, -mc)) : 0.f;
-          const float e1 = (k0 + 1 < valid) ? ex2_approx(fmaf(v[2 * t + 1], kAttnScaleLog2, -mc)) : 0.f;
-          rs += e0 + e1;
-          pk[t] = pack_bf16x2(e0, e1);
+          for (int t = 0; t < 128; ++t) s[t] = (t < valid) ? s[t] : -INFINITY;
         }
-        uint8_t* prow = sP + (c >> 1) * (AttnCfg::P_BYTES / 2) + r * 128;
+        const float mx = row_max128(s);
+        const float m_new = fmaxf(m, mx);
+        const bool resc = (m_new - m) * kAttnScaleLog2 > kRescaleLog2;
+        float alpha = 1.f;
+        if (resc) {
+          alpha = ex2_approx((m - m_new) * kAttnScaleLog2);
+          m = m_new;
+        }
+        const float mc = m * kAttnScaleLog2;
+        __syncwarp();
+        if (valid < ATT_BN)
+          softmax_block_p<true>(s, mc, valid, t_s);
+        else
+          softmax_block_p<false>(s, mc, valid, t_s);
+        if (j > 0 && __any_sync(0xffffffffu, resc)) {
+          // O_i holds the blocks before j at the old maximum: wait for the last of them, rescale.
+          if (!mbar_wait(&pv_done[wg], static_cast<uint32_t>(j - 1) & 1u, abort_flag, gstatus,
+                         DEV_TIMEOUT_ATTN + 7)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          float o[64];
+          tmem_ld64(t_o, o);
+          uint32_t ob[64];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int chunk = ((c & 1) * 4 + t) ^ (r & 7);
-          *reinterpret_cast<uint4*>(prow + chunk * 16) = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+          for (int t = 0; t < 64; ++t) ob[t] = __float_as_uint(o[t] * alpha);
+          tmem_st64(t_o, ob);
+          float o2[16];
+          tmem_ld16(t_o + 64, o2);
+          uint32_t ob2[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) ob2[t] = __float_as_uint(o2[t] * alpha);
+          tmem_st16(t_o + 64, ob2);
         }
+        tc_fence_before();
+        mbar_arrive(&p_full[wg]);
       }
-      l = fmaf(l, alpha, rs);
-      m = m_new;
-      alpha_prev = alpha;
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full);
-    }
-    if (ok && nkv > 0) {
-      const int s = (nkv - 1) & 1;
-      if (mbar_wait(&pv_full[s], static_cast<uint32_t>((nkv - 1) >> 1) & 1u, abort_flag, gstatus,
-                    DEV_TIMEOUT_ATTN + 8)) {
+      if (ok && mbar_wait(mma_done, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 8)) {
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float v[32];
-          __syncwarp();
-          tmem_ld32(lane_base + 128u + static_cast<uint32_t>(s * 64 + c * 32), v);
-#pragma unroll
-          for (int t = 0; t < 32; ++t) o[c * 32 + t] = fmaf(o[c * 32 + t], alpha_prev, v[t]);
-        }
-        const int row = qblk * ATT_BM + r;
+        float o[64], lsum[16];
+        __syncwarp();
+        tmem_ld64(t_o, o);
+        tmem_ld16(t_o + 64, lsum);
+        const int row = (tile0 + wg) * ATT_BM + r;
         if (row < T) {
-          const float inv = 1.0f / l;
+          const float inv = 1.0f / lsum[0];
           uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(b) * T + row) * D + h * 64);
 #pragma unroll
           for (int t = 0; t < 8; ++t) {

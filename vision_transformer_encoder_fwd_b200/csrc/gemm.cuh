@@ -2,16 +2,18 @@
 // (both K-contiguous, nn.Linear layout for B) and an fp32 accumulator in tensor memory,
 // followed by one of the encoder's fused epilogues.
 //
-// CTA = 6 warps, one CTA per SM, grid = min(#tiles, #SMs), tiles visited with stride gridDim:
+// CTA = 10 warps, one CTA per SM, grid = min(#tiles, #SMs), tiles visited with stride gridDim:
 //   warp 0 (one lane)  TMA producer: A tile 128 x 64 and B tile BN x 64 per stage, 128-byte
 //                      swizzle, STAGES-deep ring guarded by full/empty mbarriers.
 //   warp 1             allocates 512 TMEM columns (two BN-wide fp32 accumulators); one lane
 //                      issues tcgen05.mma (M = 128, N = BN, K = 16) four times per stage and
 //                      commits each stage back to the producer and each finished tile to
 //                      the epilogue.
-//   warps 2..5         epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, i.e. one output
-//                      row per thread, 32 columns per tcgen05.ld; applies the epilogue and
-//                      writes global memory, then releases the accumulator.
+//   warps 2..9         epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, i.e. one output
+//                      row per thread, and half of the tile's columns (warps 2..5 the first
+//                      half, 6..9 the second), 32 columns per tcgen05.ld; applies the epilogue
+//                      and writes global memory, then releases the accumulator.  Two warps per
+//                      lane quarter give each SM sub-partition two epilogue warps to overlap.
 // The double-buffered accumulator lets the epilogue of tile i overlap the MMAs of tile i+1.
 #pragma once
 
@@ -21,7 +23,8 @@ namespace vit {
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 64;
-constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_THREADS = 320;
+constexpr int GEMM_EPI_THREADS = 256;
 
 enum EpiMode : int {
   EPI_BIAS = 0,    // out_bf16 = act(acc + bias)
@@ -38,14 +41,14 @@ struct EpiParams {
   int ldo;
   // LNFOLD: per-row LayerNorm statistics rebuilt from partials written by the producer of x
   const float* colsum;     // [N] column sums of the gamma-folded weight
-  const float2* stats_in;  // [M, nt] (mean, M2) of column groups of nt_cols each
+  const float2* stats_in;  // [M, nt] (mean, M2) of column groups of nt_cols each (nt_cols = BN/2 of the producer)
   int nt, nt_cols, D;
   float eps;
   // RESID / PATCH
   float* x;              // [rows, N] fp32 residual stream
   __nv_bfloat16* xb;     // [rows, N] bf16 copy of x (A operand of the next folded GEMM)
   const float* ls;       // [N] layer scale (RESID)
-  float2* stats_out;     // [rows, N / BN] (mean, M2) over each BN-column group
+  float2* stats_out;     // [rows, N / (BN/2)] (mean, M2) over each group of BN/2 columns
   // PATCH: GEMM row m = b * P + p goes to token row b * T + 1 + R + p, position row p + pos_off
   const float* pos;
   int P, T, R, pos_off;
@@ -70,8 +73,14 @@ __device__ __forceinline__ void merge_stats(float& n, float& mean, float& m2, fl
   n = tot;
 }
 
+// One thread's part of a tile: row `row`, columns n0 .. n0 + BN/2 - 1 (TMEM columns from taddr).
+// RESID: `xpre` holds the first 32 columns of x for this row, loaded before the accumulator was
+// ready; each following chunk of x is loaded while the current one is being processed.
 template <int BN, int MODE>
-__device__ __forceinline__ void gemm_epilogue_tile(const EpiParams& ep, uint32_t taddr, int row, int n0) {
+__device__ __forceinline__ void gemm_epilogue_tile(const EpiParams& ep, uint32_t taddr, int row, int n0,
+                                                   float4 (&xpre)[8]) {
+  constexpr int HALF = BN / 2;
+  constexpr int CHUNKS = HALF / 32;
   const bool valid = row < ep.M;
   float mu = 0.f, rstd = 0.f;
   if (MODE == EPI_LNFOLD && valid) {
@@ -95,11 +104,21 @@ __device__ __forceinline__ void gemm_epilogue_tile(const EpiParams& ep, uint32_t
   float run_n = 0.f, run_mean = 0.f, run_m2 = 0.f;
 
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = 0; c < CHUNKS; ++c) {
     float v[32];
+    const int n = n0 + c * 32;
+    float4 xc[8];
+    if (MODE == EPI_RESID) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xc[j] = xpre[j];
+      if (valid && c + 1 < CHUNKS) {
+        const float4* xn = reinterpret_cast<const float4*>(ep.x + static_cast<size_t>(xrow) * ep.N + n + 32);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xpre[j] = xn[j];
+      }
+    }
     __syncwarp();
     tmem_ld32(taddr + c * 32, v);
-    const int n = n0 + c * 32;
     if (valid) {
       if (MODE == EPI_BIAS || MODE == EPI_LNFOLD) {
         const float4* b4 = reinterpret_cast<const float4*>(ep.bias + n);
@@ -146,7 +165,7 @@ __device__ __forceinline__ void gemm_epilogue_tile(const EpiParams& ep, uint32_t
           const float4* l4 = reinterpret_cast<const float4*>(ep.ls + n);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float4 xo = xp[j];
+            const float4 xo = xc[j];
             const float4 bb = __ldg(b4 + j);
             const float4 ll = __ldg(l4 + j);
             v[4 * j + 0] = fmaf(ll.x, v[4 * j + 0] + bb.x, xo.x);
@@ -193,7 +212,7 @@ __device__ __forceinline__ void gemm_epilogue_tile(const EpiParams& ep, uint32_t
     }
   }
   if ((MODE == EPI_RESID || MODE == EPI_PATCH) && valid) {
-    ep.stats_out[static_cast<size_t>(xrow) * (ep.N / BN) + n0 / BN] = make_float2(run_mean, run_m2);
+    ep.stats_out[static_cast<size_t>(xrow) * (ep.N / HALF) + n0 / HALF] = make_float2(run_mean, run_m2);
   }
 }
 
@@ -226,7 +245,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], GEMM_EPI_THREADS);
     }
     mbar_init(mma_done, 1);
     fence_mbar_init();
@@ -323,16 +342,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else if (!skip && warp >= 2) {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mb = tile / num_n;
       const int nb = tile - mb * num_n;
+      float4 xpre[8];
+      if (MODE == EPI_RESID) {
+        // this thread's first 32 columns of x, loaded while the accumulator is still being built
+        const int row0 = mb * GEMM_BM + q * 32 + lane;
+        if (row0 < M) {
+          const float4* xs = reinterpret_cast<const float4*>(ep.x + static_cast<size_t>(row0) * ep.N + nb * BN +
+                                                             half * (BN / 2));
+#pragma unroll
+          for (int j = 0; j < 8; ++j) xpre[j] = xs[j];
+        }
+      }
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 4)) break;
       tc_fence_after();
       const int row = mb * GEMM_BM + q * 32 + lane;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      gemm_epilogue_tile<BN, MODE>(ep, taddr, row, nb * BN);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN + half * (BN / 2));
+      gemm_epilogue_tile<BN, MODE>(ep, taddr, row, nb * BN + half * (BN / 2), xpre);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       acc ^= 1;

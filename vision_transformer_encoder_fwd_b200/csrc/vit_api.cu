@@ -173,13 +173,14 @@ cudaError_t launch_gemm(int bn, int mode, const CUtensorMap& a, const CUtensorMa
   }
 }
 
-cudaError_t launch_attention(const CUtensorMap& tm, int B, int T, int heads, __nv_bfloat16* out, int* st,
-                             cudaStream_t s) {
+cudaError_t launch_attention(const CUtensorMap& tm, const __nv_bfloat16* qkv, int B, int T, int heads,
+                             __nv_bfloat16* out, int* st, cudaStream_t s) {
   static std::atomic<uint64_t> attr_done{0};
   cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel, AttnCfg::SMEM_BYTES, attr_done);
   if (e != cudaSuccess) return e;
-  dim3 grid((T + ATT_BM - 1) / ATT_BM, heads, B);
-  attn_fwd_tc_kernel<<<grid, ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, T, heads * 64, out, st);
+  const int n_qtiles = (T + ATT_BM - 1) / ATT_BM;
+  dim3 grid((n_qtiles + 1) / 2, heads, B);
+  attn_fwd_tc_kernel<<<grid, ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, qkv, T, heads * 64, out, st);
   return cudaGetLastError();
 }
 
@@ -218,7 +219,7 @@ struct BlockW {
 struct vit_model {
   vit_config cfg;
   int device = 0, nsm = 1;
-  int gh = 0, gw = 0, P = 0, T = 0, K_pe = 0, Kpad = 0, bn_res = 128, nt = 1;
+  int gh = 0, gw = 0, P = 0, T = 0, K_pe = 0, Kpad = 0, bn_res = 128, stats_cols = 64, nt = 1;
   __nv_bfloat16* patch_w = nullptr;  // [D, Kpad]
   float *patch_b = nullptr, *pos = nullptr, *cls = nullptr, *reg = nullptr, *norm_w = nullptr, *norm_b = nullptr;
   CUtensorMap tm_patch;
@@ -386,7 +387,7 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs
     ++launches;
   }
   { const int ps_ = prof_open(m, VIT_K_PREFIX, s);
-  prefix_tokens_kernel<<<dim3(m->nt, 1 + R, B), 32, 0, s>>>(m->cls, m->reg, m->pos, c.pos_on_cls, T, D, m->bn_res,
+  prefix_tokens_kernel<<<dim3(m->nt, 1 + R, B), 32, 0, s>>>(m->cls, m->reg, m->pos, c.pos_on_cls, T, D, m->stats_cols,
                                                              S.x, S.xb, S.stats);
   prof_close(m, ps_, s); }
   CKL();
@@ -405,7 +406,7 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs
       ep.colsum = bw.qkv_c;
       ep.stats_in = S.stats;
       ep.nt = m->nt;
-      ep.nt_cols = m->bn_res;
+      ep.nt_cols = m->stats_cols;
       ep.D = D;
       ep.eps = c.ln_eps;
       ep.out = S.big;
@@ -416,7 +417,7 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs
       ++launches;
     }
     { const int ps_ = prof_open(m, VIT_K_ATTENTION, s);
-    CK(launch_attention(tm_qkv3, B, T, c.heads, S.attn, m->d_status, s));
+    CK(launch_attention(tm_qkv3, S.big, B, T, c.heads, S.attn, m->d_status, s));
     prof_close(m, ps_, s); }
     ++launches;
     // proj + layer scale + residual
@@ -444,7 +445,7 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs
       ep.colsum = bw.fc1_c;
       ep.stats_in = S.stats;
       ep.nt = m->nt;
-      ep.nt_cols = m->bn_res;
+      ep.nt_cols = m->stats_cols;
       ep.D = D;
       ep.eps = c.ln_eps;
       ep.out = S.big;
@@ -568,7 +569,8 @@ vit_status vit_create(const vit_config* cfg, const vit_weights* w, vit_model** o
   m->K_pe = 3 * p * p;
   m->Kpad = static_cast<int>(align_up(m->K_pe, 64));
   m->bn_res = (D % 256 == 0) ? 256 : 128;
-  m->nt = D / m->bn_res;
+  m->stats_cols = m->bn_res / 2;  // each epilogue thread covers half of a tile's columns
+  m->nt = D / m->stats_cols;
 
   cudaStream_t s;
   auto fail = [&](vit_status e) {
@@ -931,7 +933,7 @@ vit_status vit_stage_attention(const void* qkv, int32_t B, int32_t T, int32_t he
   }
   CUtensorMap tm;
   if (!tmap_qkv3d(&tm, qkv, B, T, heads * 64)) return VIT_E_CUDA;
-  CK(launch_attention(tm, B, T, heads, static_cast<__nv_bfloat16*>(out), status,
+  CK(launch_attention(tm, static_cast<const __nv_bfloat16*>(qkv), B, T, heads, static_cast<__nv_bfloat16*>(out), status,
                       reinterpret_cast<cudaStream_t>(stream)));
   return VIT_OK;
 }
