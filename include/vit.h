@@ -162,6 +162,25 @@ vit_status vit_seg_zero_shot(vit_model *m, const float *image, int32_t H, int32_
                              int32_t C, int32_t mode, int32_t side, int32_t stride, float *probs,
                              int32_t *labels, void *ws, size_t ws_bytes, vit_stream_t stream);
 
+/* The same forward as vit_forward for callers that may not allocate device memory while they
+ * run (for example a plug-in whose host owns every allocation, or a latency-critical loop in
+ * which an allocation could block or synchronise the device).  The pages have no counterpart:
+ * this entry point is an addition of this library.
+ *   The workspace comes from a fixed 64 MiB device array inside the library instead of from
+ *   the caller; images and outputs are as for vit_forward and are still the caller's.  This
+ *   entry point itself allocates nothing.
+ *   Limit: batches whose vit_workspace_size exceeds 64 MiB are rejected with VIT_E_WORKSPACE
+ *   and a message naming the size (ViT-S/16 at 336 x 336 needs about 2.8 MB per image, so up
+ *   to 24 images fit; ViT-L/16 at 1024 x 1024 needs 67.5 MB and does not fit even one image).
+ *   Every GPU that loads the library holds the 64 MiB until the process exits.
+ *   The first call on each device looks up the array's device address (cudaGetSymbolAddress)
+ *   with that device current; make that first call before any stream capture.
+ *   All calls share the one array, on every stream and model: calls whose work overlaps on
+ *   the GPU race on it and must be serialised by the caller.  Nothing in it needs to start at
+ *   zero; each call overwrites what it reads. */
+vit_status vit_forward_noalloc(vit_model *m, const float *images, int32_t B, const vit_outputs *out,
+                               vit_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the model's device status word.  Returns VIT_OK,
  * VIT_E_DEVICE_TIMEOUT if a kernel gave up on a pipeline wait since the last poll, or
  * VIT_E_CUDA if the stream reports an error. */

@@ -79,6 +79,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "vit_forward": (I32, [P, P, I32, ctypes.POINTER(VitOutputs), P, SZ, P]),
         "vit_host_workspace_size": (I32, [P, I32, ctypes.POINTER(SZ)]),
         "vit_forward_host": (I32, [P, P, I32, P, P, P, SZ, P]),
+        "vit_forward_noalloc": (I32, [P, P, I32, ctypes.POINTER(VitOutputs), P]),
         "vit_seg_workspace_size": (I32, [P, I32, I32, I32, I32, I32, I32, ctypes.POINTER(SZ)]),
         "vit_seg_zero_shot": (I32, [P, P, I32, I32, P, I32, I32, I32, I32, P, P, P, SZ, P]),
         "vit_poll": (I32, [P, P]),

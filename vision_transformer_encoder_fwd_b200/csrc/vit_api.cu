@@ -16,6 +16,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -939,3 +940,64 @@ vit_status vit_stage_attention(const void* qkv, int32_t B, int32_t T, int32_t he
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ allocation-free forward
+// Some callers may not allocate device memory at all once they are running: hosts that hand a
+// plug-in a fixed memory budget and own every allocation themselves, or latency-critical
+// loops where an allocation could block or synchronise the device.  For them
+// vit_forward_noalloc runs the same forward as vit_forward with its workspace taken from the
+// fixed array below instead of from the caller.  The array is part of the library's device
+// image, so every GPU on which the library is loaded holds it until the process exits.
+static constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(64) << 20;  // 64 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+// Device address of g_noalloc_scratch, resolved once per device (the host-side symbol is only
+// a stand-in and must never be handed to a kernel).
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+vit_status noalloc_scratch(void** ptr) {
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) {
+    set_err("device index %d out of range for the fixed scratch table", dev);
+    return VIT_E_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    CK(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return VIT_OK;
+}
+}  // namespace
+
+extern "C" vit_status vit_forward_noalloc(vit_model* m, const float* images, int32_t B, const vit_outputs* out,
+                                          vit_stream_t stream) {
+  if (!m || !images || !aligned16(images)) {
+    set_err("model or images NULL / images not 16-byte aligned");
+    return VIT_E_INVALID_ARG;
+  }
+  if (B < 1 || B > m->cfg.max_batch) {
+    set_err("batch %d outside 1..max_batch (%d)", B, m->cfg.max_batch);
+    return VIT_E_SHAPE;
+  }
+  vit_status st = check_outputs(out);
+  if (st != VIT_OK) return st;
+  const size_t need = ws_layout(m, B).total;
+  if (need > kNoAllocScratchBytes) {
+    set_err("vit_forward_noalloc: batch %d of this model needs %zu bytes of scratch, more than the fixed %zu "
+            "bytes; use vit_forward with a caller-provided workspace",
+            B, need, kNoAllocScratchBytes);
+    return VIT_E_WORKSPACE;
+  }
+  void* ws = nullptr;
+  st = noalloc_scratch(&ws);
+  if (st != VIT_OK) return st;
+  const vit_config& c = m->cfg;
+  ImgSrc src{images, 3LL * c.img_h * c.img_w, static_cast<long long>(c.img_h) * c.img_w, c.img_w, 1, 0, 0, 0};
+  return run_forward(m, src, B, out, ws, kNoAllocScratchBytes, reinterpret_cast<cudaStream_t>(stream));
+}
