@@ -100,3 +100,29 @@ def test_repeated_calls_are_deterministic_and_launch_count():
     # im2col, patch GEMM, prefix rows, 5 per block, one per tap, final LayerNorm
     assert enc.last_launch_count() == 3 + 5 * spec.depth + len(spec.taps) + 1
     enc.close()
+
+
+def test_forward_replays_from_a_cuda_graph():
+    """vit_forward enqueues only kernel launches on the caller's stream, so it can be captured into
+    a CUDA graph (the bench times small batches that way); the replay must match an eager call."""
+    need_cuda()
+    import vision_transformer_encoder_fwd_b200 as V
+    spec = S.PRESETS["small_s16"]
+    w = S.make_weights(spec, 61)
+    x = S.make_images(spec, 2, 62).cuda()
+    enc = V.VitEncoder(spec, w, max_batch=2)
+    ws = torch.empty(enc.workspace_size(2), dtype=torch.uint8, device="cuda")
+    eager = enc.forward(x, desc=True, patch=True)
+    outs = enc.alloc_outputs(2, desc=True, patch=True)
+    enc.forward_into(x, outs, ws=ws)          # warm-up outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        enc.forward_into(x, outs, ws=ws)
+    outs["desc"].zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    enc.poll()
+    assert torch.equal(outs["desc"], eager["desc"]) and torch.equal(outs["patch_tokens"], eager["patch_tokens"])
+    del g
+    enc.close()
