@@ -49,7 +49,7 @@ struct AttnCfg {
   static constexpr int OFF_ONES = OFF_V + ATT_KV_STAGES * V_BYTES;
   static constexpr int OFF_BAR = OFF_ONES + V_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 256;
-  static_assert(8 * (2 * ATT_KV_STAGES + 8) + 8 <= 256, "barrier area too small");
+  static_assert(8 * (2 * ATT_KV_STAGES + 10) + 8 <= 256, "barrier area too small");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int O_COLS = 80;                 // 64 output columns + the sum column + padding
   static constexpr uint32_t TM_S = 0, TM_O = 256, TM_Q = 416;
@@ -102,9 +102,12 @@ __device__ __forceinline__ float row_max128(const float (&s)[128]) {
 // P for one row of one key block: p = 2^(s * c - m * c) for pairs of keys (one packed fp32 FMA
 // forms the exponent pair); masked keys carry s = -inf and come out as 0 (the FMA-pipe path
 // clamps them to 2^-125 and they are zeroed explicitly).  Each 32-key chunk is packed to bf16
-// and stored to TMEM (16 columns from t_p) as soon as it is done; one wait covers the stores.
+// and stored to TMEM (16 columns from t_p).  After keys 0..63 the stores are waited for and
+// `half0` is arrived on, so the MMA can start on them while keys 64..127 are computed; `half1`
+// follows the second half.
 template <bool MASK>
-__device__ __forceinline__ void softmax_block_p(const float (&s)[128], float mc, int valid, uint32_t t_p) {
+__device__ __forceinline__ void softmax_block_p(const float (&s)[128], float mc, int valid, uint32_t t_p,
+                                                uint64_t* half0, uint64_t* half1) {
   const float2 cc = make_float2(kAttnScaleLog2, kAttnScaleLog2);
   const float2 nm = make_float2(-mc, -mc);
 #pragma unroll
@@ -127,8 +130,12 @@ __device__ __forceinline__ void softmax_block_p(const float (&s)[128], float mc,
       pk[u >> 1] = pack_bf16x2(e.x, e.y);
     }
     tmem_st16_nowait(t_p + c * 16, pk);
+    if (c == 1 || c == 3) {
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(c == 1 ? half0 : half1);
+    }
   }
-  tmem_st_wait();
 }
 
 __global__ void __launch_bounds__(ATT_THREADS, 1)
@@ -147,8 +154,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint64_t* kv_full = bars;                               // [ATT_KV_STAGES]
   uint64_t* kv_empty = kv_full + ATT_KV_STAGES;           // [ATT_KV_STAGES]
   uint64_t* s_full = kv_empty + ATT_KV_STAGES;            // [2]
-  uint64_t* p_full = s_full + 2;                          // [2]
-  uint64_t* pv_done = p_full + 2;                         // [2]
+  uint64_t* p_full = s_full + 2;                          // [2][2]: tile i, key half h at p_full[2 i + h]
+  uint64_t* pv_done = p_full + 4;                         // [2]
   uint64_t* mma_done = pv_done + 2;                       // 1
   uint64_t* q_ready = mma_done + 1;                       // 1: both Q tiles copied into TMEM
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(q_ready + 1);
@@ -172,7 +179,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[2 * i], 128);
+      mbar_init(&p_full[2 * i + 1], 128);
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(mma_done, 1);
@@ -269,12 +277,28 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 #pragma unroll
         for (int k = 0; k < 4; ++k) dk1[k] = dk0[k] + static_cast<uint64_t>(s1) * kStepK;
         for (int i = 0; i < ntile && ok; ++i) {
-          if (!mbar_wait(&p_full[i], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 4)) {
+          // P arrives in two halves of 64 keys: the first four PV MMAs run while the softmax
+          // group is still producing the second half.
+          if (!mbar_wait(&p_full[2 * i], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 4)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          tc_mma_ts_chain8(t_o0 + i * AttnCfg::O_COLS, ap[i], dvs, idesc_o, j > 0 ? 1u : 0u);
+          {
+            const uint32_t a_lo[4] = {ap[i][0], ap[i][1], ap[i][2], ap[i][3]};
+            const uint64_t b_lo[4] = {dvs[0], dvs[1], dvs[2], dvs[3]};
+            tc_mma_ts_chain4(t_o0 + i * AttnCfg::O_COLS, a_lo, b_lo, idesc_o, j > 0 ? 1u : 0u);
+          }
+          if (!mbar_wait(&p_full[2 * i + 1], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 9)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          {
+            const uint32_t a_hi[4] = {ap[i][4], ap[i][5], ap[i][6], ap[i][7]};
+            const uint64_t b_hi[4] = {dvs[4], dvs[5], dvs[6], dvs[7]};
+            tc_mma_ts_chain4(t_o0 + i * AttnCfg::O_COLS, a_hi, b_hi, idesc_o, 1u);
+          }
           tc_commit(&pv_done[i]);
           if (j + 1 < nkv) {
             if (i == 0) {
@@ -350,35 +374,32 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           alpha = ex2_approx((m - m_new) * kAttnScaleLog2);
           m = m_new;
         }
-        const float mc = m * kAttnScaleLog2;
-        __syncwarp();
-        if (valid < ATT_BN)
-          softmax_block_p<true>(s, mc, valid, t_s);
-        else
-          softmax_block_p<false>(s, mc, valid, t_s);
         if (j > 0 && __any_sync(0xffffffffu, resc)) {
-          // O_i holds the blocks before j at the old maximum: wait for the last of them, rescale.
+          // O_i holds the blocks before j at the old maximum: wait for the last of them, rescale
+          // (the sum column included) before any P of block j is released to the MMA.
           if (!mbar_wait(&pv_done[wg], static_cast<uint32_t>(j - 1) & 1u, abort_flag, gstatus,
                          DEV_TIMEOUT_ATTN + 7)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          float o[64];
-          tmem_ld64(t_o, o);
-          uint32_t ob[64];
+          // 16 columns at a time: the 128 logits stay live in registers meanwhile
+#pragma unroll 1
+          for (int c = 0; c < AttnCfg::O_COLS; c += 16) {
+            float o[16];
+            tmem_ld16(t_o + c, o);
+            uint32_t ob[16];
 #pragma unroll
-          for (int t = 0; t < 64; ++t) ob[t] = __float_as_uint(o[t] * alpha);
-          tmem_st64(t_o, ob);
-          float o2[16];
-          tmem_ld16(t_o + 64, o2);
-          uint32_t ob2[16];
-#pragma unroll
-          for (int t = 0; t < 16; ++t) ob2[t] = __float_as_uint(o2[t] * alpha);
-          tmem_st16(t_o + 64, ob2);
+            for (int t = 0; t < 16; ++t) ob[t] = __float_as_uint(o[t] * alpha);
+            tmem_st16(t_o + c, ob);
+          }
         }
-        tc_fence_before();
-        mbar_arrive(&p_full[wg]);
+        const float mc = m * kAttnScaleLog2;
+        __syncwarp();
+        if (valid < ATT_BN)
+          softmax_block_p<true>(s, mc, valid, t_s, &p_full[2 * wg], &p_full[2 * wg + 1]);
+        else
+          softmax_block_p<false>(s, mc, valid, t_s, &p_full[2 * wg], &p_full[2 * wg + 1]);
       }
       if (ok && mbar_wait(mma_done, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 8)) {
         tc_fence_after();
