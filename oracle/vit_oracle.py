@@ -52,10 +52,10 @@ import numpy as np
 from scipy.special import erf as _erf
 
 __all__ = [
-    "bf16_round", "to_f64_weights", "patch_embed", "assemble_tokens", "layer_norm", "gelu",
+    "bicubic_resize", "resize_pos_embed", "bf16_round", "to_f64_weights", "patch_embed", "assemble_tokens", "layer_norm", "gelu",
     "attention", "attention_probs", "encoder_block", "forward", "l2_normalize", "cos_map",
     "bilinear_resize", "window_origins", "overlap_counts", "seg_slide_from_tokens",
-    "seg_whole_from_tokens", "seg_slide", "HEAD_DIM",
+    "seg_whole_from_tokens", "seg_slide", "seg_whole", "text_head", "HEAD_DIM",
 ]
 
 HEAD_DIM = 64
@@ -90,6 +90,54 @@ def to_f64_weights(weights) -> Dict[str, object]:
     out = {k: conv(v) for k, v in weights.items() if k != "blocks"}
     out["blocks"] = [{k: conv(v) for k, v in b.items()} for b in weights["blocks"]]
     return out
+
+
+# ---------------------------------------------------------------------------------------------
+# [diagram] "DINOv2-S encoder": "Position embedding 1,370 x 384" followed by "Bicubic
+# interpolation, 37x37 unchanged" -- the learned grid is resized bicubically to the input's
+# patch grid (the identity at the native size).  Reading: the convolution form of bicubic
+# interpolation with a = -0.75, half-pixel centres (align_corners=False), source coordinates
+# not clamped, taps clamped to the border -- the convention of F.interpolate(mode="bicubic").
+# ---------------------------------------------------------------------------------------------
+def _cubic_weights(t: np.ndarray, a: float = -0.75) -> np.ndarray:
+    """Weights of the taps at offsets -1, 0, +1, +2 for fractional positions t in [0, 1)."""
+    def k(x):
+        x = np.abs(x)
+        return np.where(x <= 1.0, ((a + 2.0) * x - (a + 3.0)) * x * x + 1.0,
+                        np.where(x < 2.0, ((a * x - 5.0 * a) * x + 8.0 * a) * x - 4.0 * a, 0.0))
+    return np.stack([k(1.0 + t), k(t), k(1.0 - t), k(2.0 - t)], axis=-1)
+
+
+def bicubic_resize(img: np.ndarray, out_h: int, out_w: int) -> np.ndarray:
+    """[C, h, w] -> [C, out_h, out_w], separable: rows, then columns."""
+    C, h, w = img.shape
+
+    def axis(n_in, n_out):
+        src = (np.arange(n_out, dtype=np.float64) + 0.5) * (n_in / n_out) - 0.5
+        i0 = np.floor(src).astype(np.int64)
+        wts = _cubic_weights(src - i0)
+        idx = np.clip(i0[:, None] + np.arange(-1, 3)[None, :], 0, n_in - 1)
+        return idx, wts
+
+    ry, wy = axis(h, out_h)
+    rx, wx = axis(w, out_w)
+    rows = (img[:, ry, :] * wy[None, :, :, None]).sum(axis=2)           # [C, out_h, w]
+    return (rows[:, :, rx] * wx[None, None, :, :]).sum(axis=3)
+
+
+def resize_pos_embed(pos: np.ndarray, grid0, grid, pos_on_cls: bool) -> np.ndarray:
+    """Position embedding for a patch grid `grid` from the learned one for `grid0`: the patch rows
+    are resized bicubically as a [D, gh0, gw0] image; a CLS row (pos_on_cls) is kept as is."""
+    gh0, gw0 = grid0
+    gh, gw = grid
+    cls = pos[:1] if pos_on_cls else pos[:0]
+    patch = pos[(1 if pos_on_cls else 0):]
+    if (gh, gw) == (gh0, gw0):
+        return pos.copy()
+    D = patch.shape[1]
+    img = patch.reshape(gh0, gw0, D).transpose(2, 0, 1)
+    out = bicubic_resize(img, gh, gw).transpose(1, 2, 0).reshape(gh * gw, D)
+    return np.concatenate([cls, out], axis=0)
 
 
 # ---------------------------------------------------------------------------------------------
@@ -212,11 +260,13 @@ def forward(images, weights, spec, n_blocks: Optional[int] = None, record_hidden
             ) -> Dict[str, object]:
     """The encoder forward of ``spec`` on fp32 images [B, 3, H, W].
 
-    Steps: bf16 rounding of the input; patch embedding; CLS / register / position tokens;
+    Steps: bf16 rounding of the input; patch embedding; CLS / register / position tokens (the
+    learned grid resized bicubically when the input's patch grid differs from the native one);
     ``depth`` encoder blocks (taps after the blocks listed in ``spec.taps``); final
     LayerNorm; outputs
       desc          [B, D]   L2-normalised final-norm CLS token ([card] "Usage")
       patch_tokens  [B, P, D] final-norm tokens of the patches (CLS and registers dropped)
+      final_tokens  [B, T, D] the whole final-norm sequence (CLS, registers, patches)
       taps          {l: [B, D, gh, gw]} final-norm tokens after block l, CLS and registers
                     removed, channels first ([diagram] "Tap stage", "Taps apply LayerNorm,
                     remove CLS, reshape")
@@ -234,7 +284,8 @@ def forward(images, weights, spec, n_blocks: Optional[int] = None, record_hidden
     gh, gw = xb.shape[2] // p, xb.shape[3] // p
     P = gh * gw
     e = patch_embed(xb, w["patch_w"], w["patch_b"], p)
-    x = assemble_tokens(e, w["cls"], w["reg"] if R else None, w["pos"], spec.pos_on_cls)
+    pos = resize_pos_embed(w["pos"], (spec.grid_h, spec.grid_w), (gh, gw), spec.pos_on_cls)
+    x = assemble_tokens(e, w["cls"], w["reg"] if R else None, pos, spec.pos_on_cls)
     L = spec.depth if n_blocks is None else n_blocks
     hidden = np.empty((L, B, x.shape[1], D)) if record_hidden else None
     taps: Dict[int, np.ndarray] = {}
@@ -253,6 +304,7 @@ def forward(images, weights, spec, n_blocks: Optional[int] = None, record_hidden
         "desc": l2_normalize(n[:, 0, :]),
         "cls_norm": n[:, 0, :].copy(),
         "patch_tokens": n[:, 1 + R:, :].copy(),
+        "final_tokens": n,
         "taps": taps,
         "grid": (gh, gw),
     }
@@ -343,6 +395,26 @@ def seg_slide_from_tokens(window_tokens: np.ndarray, text: np.ndarray, H: int, W
     return probs, np.argmax(probs, axis=0)
 
 
+# ---------------------------------------------------------------------------------------------
+# [dino.txt article] "Aligning 1024-d patch tokens with 2048-d text embeddings": on the vision
+# side the backbone's 1024-d patch tokens first go through 2 extra self-attention blocks
+# (vision_model_num_head_blocks = 2), then meet the patch half of the text embedding in a
+# cosine.  Readings: each head block has the encoder block's form and width (pre-LN attention
+# and MLP branches with layer scale); it runs on the backbone's whole final-norm sequence
+# (CLS, registers and patches attend to one another as in the backbone); the head's patch rows
+# go to the cosine as they come out of the last block (the passage names no further norm, and
+# the cosine divides by the token's length anyway).
+# ---------------------------------------------------------------------------------------------
+def text_head(final_tokens: np.ndarray, head_blocks, spec) -> np.ndarray:
+    """final_tokens [B, T, D] (backbone final-norm sequence) -> head patch tokens [B, P, D]."""
+    hb = to_f64_weights({"blocks": head_blocks})["blocks"]
+    x = np.array(final_tokens, dtype=np.float64, copy=True)
+    for bw in hb:
+        for i in range(x.shape[0]):
+            x[i] = encoder_block(x[i], bw, spec.heads, spec.ln_eps)
+    return x[:, 1 + spec.registers:, :].copy()
+
+
 def seg_whole_from_tokens(tokens: np.ndarray, text: np.ndarray, H: int, W: int,
                           grid: Tuple[int, int]) -> Tuple[np.ndarray, np.ndarray]:
     """predict_whole: cos map [C, h, w] upsampled bilinearly to [C, H, W]; argmax."""
@@ -350,9 +422,12 @@ def seg_whole_from_tokens(tokens: np.ndarray, text: np.ndarray, H: int, W: int,
     return up, np.argmax(up, axis=0)
 
 
-def seg_slide(image, weights, spec, text, side: int, stride: int, n_windows: Optional[int] = None):
+def seg_slide(image, weights, spec, text, side: int, stride: int, n_windows: Optional[int] = None,
+              head_blocks=None):
     """Full slide mode on one image [3, H, W] (or [1, 3, H, W]): crops every window, runs the
-    encoder of ``spec`` (whose input size must be side x side) on each, then scores.
+    encoder of ``spec`` on each (its position grid resized to side/p x side/p when the window is
+    not the size it was learned for) and, if ``head_blocks`` is given, the dino.txt vision head
+    (text_head), then scores.
     Returns (probs, labels, window_tokens)."""
     img = image.detach().cpu().numpy() if hasattr(image, "detach") else np.asarray(image)
     if img.ndim == 4:
@@ -367,7 +442,21 @@ def seg_slide(image, weights, spec, text, side: int, stride: int, n_windows: Opt
     w = to_f64_weights(weights) if not isinstance(weights.get("patch_w"), np.ndarray) else weights
     toks = []
     for i in range(crops.shape[0]):
-        toks.append(forward(crops[i:i + 1], w, spec)["patch_tokens"][0])
+        o = forward(crops[i:i + 1], w, spec)
+        toks.append(o["patch_tokens"][0] if head_blocks is None else text_head(o["final_tokens"], head_blocks, spec)[0])
     toks = np.stack(toks)
     probs, labels = seg_slide_from_tokens(toks, txt, H, W, side, stride, (side // spec.patch, side // spec.patch))
     return probs, labels, toks
+
+
+def seg_whole(image, weights, spec, text, head_blocks=None):
+    """Whole mode on one image [3, H, W]: one encoder pass at the image's own size (position grid
+    resized as in forward), the dino.txt head if given, then seg_whole_from_tokens."""
+    img = image.detach().cpu().numpy() if hasattr(image, "detach") else np.asarray(image)
+    if img.ndim == 3:
+        img = img[None]
+    txt = text.detach().double().cpu().numpy() if hasattr(text, "detach") else np.asarray(text, np.float64)
+    o = forward(img, weights, spec)
+    tok = o["patch_tokens"][0] if head_blocks is None else text_head(o["final_tokens"], head_blocks, spec)[0]
+    scores, labels = seg_whole_from_tokens(tok, txt, img.shape[2], img.shape[3], o["grid"])
+    return scores, labels, tok

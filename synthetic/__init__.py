@@ -80,13 +80,21 @@ VITS14_518 = ModelSpec("vits14_518", 14, 518, 518, 384, 12, 6, 1536, 0, True, (3
 VITL16_1024 = ModelSpec("vitl16_1024", 16, 1024, 1024, 1024, 24, 16, 4096, 4, False)
 VITL16_384 = ModelSpec("vitl16_384", 16, 384, 384, 1024, 24, 16, 4096, 4, False)
 
+# Other widths of the DINOv2 family ("DINOv2模型服务" blog, model-variant table: ViT-B/14
+# 768 / 12 blocks / 12 heads, ViT-G/14 1536 / 40 / 24), DINOv2-style (no registers, position
+# embedding on CLS), MLP ratio 4 with GELU as in the blog's DinoVisionTransformer(mlp_ratio=4);
+# at 224 x 224 (16 x 16 patches, 257 tokens) so the fp64 oracle stays fast.
+VITB14_224 = ModelSpec("vitb14_224", 14, 224, 224, 768, 12, 12, 3072, 0, True)
+VITG14_224 = ModelSpec("vitg14_224", 14, 224, 224, 1536, 40, 24, 6144, 0, True)
+
 # Small shapes for fast parity runs (several GEMM tiles and a ragged tail, seconds in fp64).
 TINY_S16 = ModelSpec("tiny_s16", 16, 96, 160, 128, 2, 2, 512, 4, False)            # T = 65
 TINY_S14 = ModelSpec("tiny_s14", 14, 126, 126, 128, 3, 2, 256, 0, True, (1, 3))     # T = 82
 SMALL_S16 = ModelSpec("small_s16", 16, 224, 224, 256, 3, 4, 1024, 4, False, (2,))   # T = 201
 
 PRESETS: Dict[str, ModelSpec] = {
-    s.name: s for s in (VITS16_336, VITS14_518, VITL16_1024, VITL16_384, TINY_S16, TINY_S14, SMALL_S16)
+    s.name: s for s in (VITS16_336, VITS14_518, VITL16_1024, VITL16_384, VITB14_224, VITG14_224, TINY_S16, TINY_S14,
+                        SMALL_S16)
 }
 
 
@@ -116,6 +124,10 @@ SLIDE_SIDE = 384
 SLIDE_STRIDE = 192
 SLIDE_CLASSES = 150
 TEXT_SEED = 5150
+# dino.txt vision head: 2 extra blocks on the backbone's tokens before the cosine with the
+# text features (dino.txt article, "Aligning 1024-d patch tokens with 2048-d text embeddings").
+DINOTXT_HEAD_BLOCKS = 2
+HEAD_SEED = 5151
 
 
 def to_bf16(t: torch.Tensor) -> torch.Tensor:
@@ -129,6 +141,26 @@ def _normal(g: torch.Generator, shape, std: float) -> torch.Tensor:
 
 def _uniform(g: torch.Generator, shape, lo: float, hi: float) -> torch.Tensor:
     return lo + (hi - lo) * torch.rand(*shape, generator=g, dtype=torch.float32)
+
+
+def _block_weights(g: torch.Generator, D: int, F: int) -> Dict[str, torch.Tensor]:
+    """One encoder block's weights in draw order (qkv left fp32 for the sink construction)."""
+    return {
+        "ln1_w": to_bf16(1.0 + _normal(g, (D,), 0.02)),
+        "ln1_b": to_bf16(_normal(g, (D,), 0.02)),
+        "qkv_w": _normal(g, (3 * D, D), 0.02),
+        "qkv_b": _normal(g, (3 * D,), 0.02),
+        "proj_w": to_bf16(_normal(g, (D, D), 0.02)),
+        "proj_b": to_bf16(_normal(g, (D,), 0.02)),
+        "ls1": to_bf16(_uniform(g, (D,), 0.1, 1.0)),
+        "ln2_w": to_bf16(1.0 + _normal(g, (D,), 0.02)),
+        "ln2_b": to_bf16(_normal(g, (D,), 0.02)),
+        "fc1_w": to_bf16(_normal(g, (F, D), 0.02)),
+        "fc1_b": to_bf16(_normal(g, (F,), 0.02)),
+        "fc2_w": to_bf16(_normal(g, (D, F), 0.02)),
+        "fc2_b": to_bf16(_normal(g, (D,), 0.02)),
+        "ls2": to_bf16(_uniform(g, (D,), 0.1, 1.0)),
+    }
 
 
 def make_weights(spec: ModelSpec, seed: int, outlier: bool = False) -> Dict[str, object]:
@@ -151,25 +183,7 @@ def make_weights(spec: ModelSpec, seed: int, outlier: bool = False) -> Dict[str,
     w["pos"] = to_bf16(_normal(g, (spec.n_pos, D), 0.02))
     w["norm_w"] = to_bf16(1.0 + _normal(g, (D,), 0.02))
     w["norm_b"] = to_bf16(_normal(g, (D,), 0.02))
-    blocks: List[Dict[str, torch.Tensor]] = []
-    for _ in range(spec.depth):
-        b = {
-            "ln1_w": to_bf16(1.0 + _normal(g, (D,), 0.02)),
-            "ln1_b": to_bf16(_normal(g, (D,), 0.02)),
-            "qkv_w": _normal(g, (3 * D, D), 0.02),
-            "qkv_b": _normal(g, (3 * D,), 0.02),
-            "proj_w": to_bf16(_normal(g, (D, D), 0.02)),
-            "proj_b": to_bf16(_normal(g, (D,), 0.02)),
-            "ls1": to_bf16(_uniform(g, (D,), 0.1, 1.0)),
-            "ln2_w": to_bf16(1.0 + _normal(g, (D,), 0.02)),
-            "ln2_b": to_bf16(_normal(g, (D,), 0.02)),
-            "fc1_w": to_bf16(_normal(g, (F, D), 0.02)),
-            "fc1_b": to_bf16(_normal(g, (F,), 0.02)),
-            "fc2_w": to_bf16(_normal(g, (D, F), 0.02)),
-            "fc2_b": to_bf16(_normal(g, (D,), 0.02)),
-            "ls2": to_bf16(_uniform(g, (D,), 0.1, 1.0)),
-        }
-        blocks.append(b)
+    blocks: List[Dict[str, torch.Tensor]] = [_block_weights(g, D, F) for _ in range(spec.depth)]
     if outlier:
         _inject_attention_sink(spec, w, blocks, seed)
     for b in blocks:
@@ -177,6 +191,17 @@ def make_weights(spec: ModelSpec, seed: int, outlier: bool = False) -> Dict[str,
         b["qkv_b"] = to_bf16(b["qkv_b"]) if b["qkv_b"].dtype != torch.bfloat16 else b["qkv_b"]
     w["blocks"] = blocks
     return w
+
+
+def make_head_weights(spec: ModelSpec, seed: int, n_blocks: int = DINOTXT_HEAD_BLOCKS) -> List[Dict[str, torch.Tensor]]:
+    """Seeded bf16 weights of the dino.txt vision head: ``n_blocks`` blocks of the encoder
+    block's form and width, drawn like make_weights' blocks."""
+    g = torch.Generator().manual_seed(int(seed))
+    blocks = [_block_weights(g, spec.dim, spec.mlp) for _ in range(n_blocks)]
+    for b in blocks:
+        b["qkv_w"] = to_bf16(b["qkv_w"])
+        b["qkv_b"] = to_bf16(b["qkv_b"])
+    return blocks
 
 
 # Attention-sink construction (kornia/dinov3 card, "Build BF16, not FP16": the scaled logits

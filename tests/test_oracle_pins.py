@@ -22,13 +22,18 @@ GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "page_
 
 
 # ------------------------------------------------------------------ independent torch composition
-def torch_forward(images, weights, spec, record_hidden=False):
+def torch_forward(images, weights, spec, record_hidden=False, head_blocks=None):
     """The encoder written with torch fp64 functional ops (F.conv2d, F.layer_norm, F.linear,
     F.scaled_dot_product_attention, F.gelu, F.normalize) -- shares no code with the oracle."""
     x = images.to(torch.bfloat16).double()
     W = {k: v.double() for k, v in weights.items() if k != "blocks"}
     e = F.conv2d(x, W["patch_w"], W["patch_b"], stride=spec.patch)
-    B, D = e.shape[0], e.shape[1]
+    B, D, gh, gw = e.shape
+    if (gh, gw) != (spec.grid_h, spec.grid_w):
+        start = 1 if spec.pos_on_cls else 0
+        grid = W["pos"][start:].reshape(1, spec.grid_h, spec.grid_w, D).permute(0, 3, 1, 2)
+        grid = F.interpolate(grid, size=(gh, gw), mode="bicubic", align_corners=False)
+        W["pos"] = torch.cat([W["pos"][:start], grid.permute(0, 2, 3, 1).reshape(gh * gw, D)])
     e = e.flatten(2).transpose(1, 2)
     parts = [W["cls"].view(1, 1, D).expand(B, 1, D)]
     if spec.registers:
@@ -42,20 +47,29 @@ def torch_forward(images, weights, spec, record_hidden=False):
     T = h.shape[1]
     hidden = []
     for bw in weights["blocks"]:
-        b = {k: v.double() for k, v in bw.items()}
-        u = F.layer_norm(h, (D,), b["ln1_w"], b["ln1_b"], spec.ln_eps)
-        qkv = F.linear(u, b["qkv_w"], b["qkv_b"]).view(B, T, 3, spec.heads, 64).permute(2, 0, 3, 1, 4)
-        o = F.scaled_dot_product_attention(qkv[0], qkv[1], qkv[2])
-        o = o.transpose(1, 2).reshape(B, T, D)
-        h = h + b["ls1"] * F.linear(o, b["proj_w"], b["proj_b"])
-        u2 = F.layer_norm(h, (D,), b["ln2_w"], b["ln2_b"], spec.ln_eps)
-        h = h + b["ls2"] * F.linear(F.gelu(F.linear(u2, b["fc1_w"], b["fc1_b"])), b["fc2_w"], b["fc2_b"])
+        h = torch_block(h, bw, spec)
         hidden.append(h.clone())
     n = F.layer_norm(h, (D,), W["norm_w"], W["norm_b"], spec.ln_eps)
     out = {"desc": F.normalize(n[:, 0], dim=-1).numpy(), "patch_tokens": n[:, 1 + spec.registers:].numpy()}
     if record_hidden:
         out["hidden"] = torch.stack(hidden).numpy()
+    if head_blocks is not None:
+        for bw in head_blocks:
+            n = torch_block(n, bw, spec)
+        out["head_tokens"] = n[:, 1 + spec.registers:].numpy()
     return out
+
+
+def torch_block(h, bw, spec):
+    B, T, D = h.shape
+    b = {k: v.double() for k, v in bw.items()}
+    u = F.layer_norm(h, (D,), b["ln1_w"], b["ln1_b"], spec.ln_eps)
+    qkv = F.linear(u, b["qkv_w"], b["qkv_b"]).view(B, T, 3, spec.heads, 64).permute(2, 0, 3, 1, 4)
+    o = F.scaled_dot_product_attention(qkv[0], qkv[1], qkv[2])
+    o = o.transpose(1, 2).reshape(B, T, D)
+    h = h + b["ls1"] * F.linear(o, b["proj_w"], b["proj_b"])
+    u2 = F.layer_norm(h, (D,), b["ln2_w"], b["ln2_b"], spec.ln_eps)
+    return h + b["ls2"] * F.linear(F.gelu(F.linear(u2, b["fc1_w"], b["fc1_b"])), b["fc2_w"], b["fc2_b"])
 
 
 def _close(a, b, rtol=1e-9):
@@ -373,6 +387,90 @@ def test_cos_map_is_cosine():
     cm = O.cos_map(toks, text, 2, 3)
     ref = torch.nn.functional.cosine_similarity(torch.from_numpy(text)[:, None, :], torch.from_numpy(toks)[None], dim=-1)
     assert _close(cm.reshape(4, 6), ref.numpy(), 1e-14)
+
+
+# ------------------------------------------------------------------ position-embedding resize
+@pytest.mark.parametrize("h,w,oh,ow", [(21, 21, 32, 64), (24, 24, 16, 40), (5, 7, 11, 3), (4, 4, 1, 1)])
+def test_bicubic_matches_interpolate(h, w, oh, ow):
+    x = torch.randn(3, h, w, generator=torch.Generator().manual_seed(h + w), dtype=torch.float64)
+    ref = F.interpolate(x[None], size=(oh, ow), mode="bicubic", align_corners=False)[0].numpy()
+    assert _close(O.bicubic_resize(x.numpy(), oh, ow), ref, 1e-13)
+
+
+def test_bicubic_identity_at_native_grid():
+    # "DINOv2 n semantic" diagram: "Bicubic interpolation, 37x37 unchanged"
+    g = GOLDEN["vits14_518"]["conv_out"][1]
+    x = np.random.default_rng(30).standard_normal((5, g, g))
+    assert np.array_equal(O.bicubic_resize(x, g, g), x)
+    pos = np.random.default_rng(31).standard_normal((1 + g * g, 8))
+    assert np.array_equal(O.resize_pos_embed(pos, (g, g), (g, g), True), pos)
+
+
+def test_resize_keeps_cls_row_and_constant_fields():
+    pos = np.random.default_rng(32).standard_normal((1 + 6 * 6, 4))
+    pos[1:] = 2.5                                   # a constant grid stays constant (weights sum to 1)
+    r = O.resize_pos_embed(pos, (6, 6), (9, 4), pos_on_cls=True)
+    assert r.shape == (1 + 36, 4) and np.array_equal(r[0], pos[0]) and np.abs(r[1:] - 2.5).max() < 1e-14
+
+
+@pytest.mark.parametrize("name,hw", [("tiny_s16", (128, 128)), ("tiny_s14", (98, 154))])
+def test_forward_at_other_sizes_matches_torch_composition(name, hw):
+    spec = S.PRESETS[name]
+    w = S.make_weights(spec, 33)
+    im = S.make_images(spec, 2, 34, *hw)
+    ours = O.forward(im, w, spec, record_hidden=True)
+    ref = torch_forward(im, w, spec, record_hidden=True)
+    assert _close(ours["hidden"], ref["hidden"], 1e-10) and _close(ours["desc"], ref["desc"], 1e-10)
+
+
+def test_planted_cubic_coefficient_mistake_is_caught(monkeypatch):
+    # a = -0.5 (Catmull-Rom) instead of the -0.75 kernel: a plausible slip the pin must see
+    orig = OV._cubic_weights
+    x = np.random.default_rng(35).standard_normal((2, 21, 21))
+    ref = F.interpolate(torch.from_numpy(x)[None], size=(32, 64), mode="bicubic", align_corners=False)[0].numpy()
+    monkeypatch.setattr(OV, "_cubic_weights", lambda t, a=-0.5: orig(t, -0.5))
+    assert not _close(OV.bicubic_resize(x, 32, 64), ref, 1e-6)
+
+
+# ------------------------------------------------------------------ dino.txt vision head
+@pytest.mark.parametrize("name,hw", [("tiny_s16", None), ("tiny_s14", (98, 154))])
+def test_text_head_matches_torch_composition(name, hw):
+    spec = S.PRESETS[name]
+    w = S.make_weights(spec, 41)
+    head = S.make_head_weights(spec, 42)
+    im = S.make_images(spec, 2, 43, *(hw or (spec.img_h, spec.img_w)))
+    o = O.forward(im, w, spec)
+    ours = O.text_head(o["final_tokens"], head, spec)
+    ref = torch_forward(im, w, spec, head_blocks=head)["head_tokens"]
+    assert len(head) == 2 and ours.shape == ref.shape == o["patch_tokens"].shape
+    assert _close(ours, ref, 1e-10)
+
+
+def test_text_head_with_zero_layer_scale_is_the_identity():
+    spec = S.PRESETS["tiny_s16"]
+    w = S.make_weights(spec, 44)
+    head = S.make_head_weights(spec, 45)
+    for b in head:
+        b["ls1"] = torch.zeros_like(b["ls1"])
+        b["ls2"] = torch.zeros_like(b["ls2"])
+    o = O.forward(S.make_images(spec, 1, 46), w, spec)
+    assert np.array_equal(O.text_head(o["final_tokens"], head, spec), o["patch_tokens"])
+
+
+def test_seg_whole_with_head_uses_head_tokens():
+    spec = S.PRESETS["tiny_s16"]
+    w = S.make_weights(spec, 47)
+    head = S.make_head_weights(spec, 48)
+    im = S.make_images(spec, 1, 49)[0]
+    text = S.make_text_feats(7, spec.dim, 50)
+    scores, labels, tok = O.seg_whole(im, w, spec, text, head_blocks=head)
+    ref = torch_forward(im[None], w, spec, head_blocks=head)["head_tokens"][0]
+    assert _close(tok, ref, 1e-10)
+    t = ref / np.linalg.norm(ref, axis=1, keepdims=True)
+    cos = (text.double().numpy() @ t.T).reshape(7, spec.grid_h, spec.grid_w)
+    up = F.interpolate(torch.from_numpy(cos)[None], size=(spec.img_h, spec.img_w), mode="bilinear",
+                       align_corners=False)[0].numpy()
+    assert _close(scores, up, 1e-10) and np.array_equal(labels, up.argmax(0))
 
 
 # ------------------------------------------------------------------ planted mistakes
