@@ -138,19 +138,58 @@ vit_status vit_host_workspace_size(const vit_model *m, int32_t batch, size_t *by
 vit_status vit_forward_host(vit_model *m, const float *images_host, int32_t B, float *desc_host,
                             void *patch_tokens_host, void *ws, size_t ws_bytes, vit_stream_t stream);
 
+/* The encoder forward at an input size other than the one the model was created for
+ * ([diagram] "DINOv2-S encoder": the learned position grid goes through "Bicubic
+ * interpolation" to the input's patch grid, the identity at the native size).
+ *   images  device fp32 [B, 3, H, W], ImageNet-normalised; patch <= H, W <= 16384.
+ *   The patch grid is gh = floor(H / patch) by gw = floor(W / patch) (the stride-p
+ *   convolution's; pixels past gh*patch, gw*patch are not read); T = 1 + R + gh*gw tokens.
+ *   At a grid other than the native one, the first kernel writes the patch rows of the position
+ *   embedding resized by separable cubic convolution (Keys' kernel, a = -0.75, half-pixel
+ *   centres, taps clamped to the border; the CLS row, if any, copied) into the workspace.
+ *   Outputs are sized by that grid: patch_tokens and taps [B, gh*gw, D], hidden [depth, B, T, D].
+ *   ws  at least vit_workspace_size_hw(m, B, H, W) bytes, 256-byte aligned.
+ * At the native size this is vit_forward.  Errors as vit_forward; VIT_E_SHAPE for H or W out of
+ * range or B * T >= 2^30.  Enqueues on `stream`. */
+vit_status vit_workspace_size_hw(const vit_model *m, int32_t batch, int32_t H, int32_t W, size_t *bytes);
+vit_status vit_forward_hw(vit_model *m, const float *images, int32_t B, int32_t H, int32_t W,
+                          const vit_outputs *out, void *ws, size_t ws_bytes, vit_stream_t stream);
+
+/* dino.txt vision head ([dinotxt] "Aligning 1024-d patch tokens with 2048-d text embeddings":
+ * the backbone's patch tokens pass through 2 extra self-attention blocks before the cosine
+ * with the text features).  Each head block has the encoder block's form and width and takes
+ * vit_block_weights like the backbone's; the head runs on the backbone's whole final-norm
+ * sequence (CLS, registers, patches) and its patch rows, as the last block leaves them, are
+ * the tokens the zero-shot scoring uses.
+ *   vit_set_text_head: attaches n_blocks (1..8) head blocks, once per model (a second call
+ *   returns VIT_E_INVALID_ARG); the weights are read as vit_create reads the backbone's (the
+ *   folded QKV/FC1 copies are made now; proj_w and fc2_w are borrowed and must stay valid).
+ *   Call it with the model's device current.  Once attached, vit_seg_zero_shot scores the
+ *   head's tokens instead of the backbone's final-norm patch tokens.
+ *   vit_forward_text_tokens: backbone + head on B images of H x W (any size as for
+ *   vit_forward_hw; workspace vit_workspace_size_hw(m, B, H, W)); tokens: device fp32
+ *   [B, floor(H/p) * floor(W/p), D].  VIT_E_INVALID_ARG if no head is attached. */
+vit_status vit_set_text_head(vit_model *m, const vit_block_weights *blocks, int32_t n_blocks);
+vit_status vit_forward_text_tokens(vit_model *m, const float *images, int32_t B, int32_t H, int32_t W,
+                                   float *tokens, void *ws, size_t ws_bytes, vit_stream_t stream);
+
 /* Zero-shot dense scoring ([dinotxt] patch/text alignment; whole and slide modes). */
 enum { VIT_SEG_WHOLE = 0, VIT_SEG_SLIDE = 1 };
 
-/* Workspace for vit_seg_zero_shot with these arguments. */
+/* Workspace for vit_seg_zero_shot with these arguments (VIT_E_SHAPE / VIT_E_INVALID_ARG for
+ * arguments vit_seg_zero_shot would reject). */
 vit_status vit_seg_workspace_size(const vit_model *m, int32_t H, int32_t W, int32_t C, int32_t mode,
                                   int32_t side, int32_t stride, size_t *bytes);
 
 /* image  device fp32 [3, H, W], ImageNet-normalised.
  * text   device fp32 [C, D] class embeddings (unit rows; used as given).
- * WHOLE: H, W must equal the model's img_h, img_w (the position embedding is not resized);
- *        the encoder runs once; scores = bilinear (align_corners=False) upsample of the cosine
- *        map cos[c, i] = text[c] . t_i / max(||t_i||, 1e-12) over the final-LN patch tokens t.
- * SLIDE: side must equal img_h == img_w; windows of side x side at `stride`, per axis
+ * Tokens: the backbone's final-norm patch tokens, or the text head's (vit_set_text_head).
+ * WHOLE: the encoder runs once on the H x W image (as vit_forward_hw: any H, W >= patch, the
+ *        position embedding resized to the floor(H/p) x floor(W/p) grid); scores = bilinear
+ *        (align_corners=False) upsample to H x W of the cosine map
+ *        cos[c, i] = text[c] . t_i / max(||t_i||, 1e-12) over the final-LN patch tokens t.
+ * SLIDE: side >= patch and side <= H, W (windows at a side other than the model's img_h x img_w
+ *        use the resized position embedding); windows of side x side at `stride`, per axis
  *        ceil((size - side) / stride) + 1 origins with the last clamped to size - side; every
  *        window runs the encoder (all windows in one batch, so max_batch must cover them);
  *        per window the cosine map is upsampled to side x side, softmaxed over classes and
@@ -186,7 +225,7 @@ vit_status vit_forward_noalloc(vit_model *m, const float *images, int32_t B, con
  * VIT_E_CUDA if the stream reports an error. */
 vit_status vit_poll(vit_model *m, vit_stream_t stream);
 
-/* Number of kernel launches the last vit_forward / vit_seg_zero_shot call made. */
+/* Number of kernel launches the last vit_forward / vit_forward_hw / vit_seg_zero_shot call made. */
 int32_t vit_last_launch_count(const vit_model *m);
 
 /* Per-launch timing on the caller's stream.  After vit_profile_begin(m, capacity) every kernel
@@ -197,7 +236,7 @@ int32_t vit_last_launch_count(const vit_model *m);
 enum {
   VIT_K_IM2COL = 0, VIT_K_PATCH_GEMM, VIT_K_PREFIX, VIT_K_QKV_GEMM, VIT_K_ATTENTION, VIT_K_PROJ_GEMM,
   VIT_K_FC1_GEMM, VIT_K_FC2_GEMM, VIT_K_TAP, VIT_K_FINAL_LN, VIT_K_SEG_NORM, VIT_K_SEG_COS, VIT_K_SEG_MAP,
-  VIT_K_COUNT
+  VIT_K_POS_RESIZE, VIT_K_HEAD_OUT, VIT_K_COUNT
 };
 vit_status vit_profile_begin(vit_model *m, int32_t capacity);
 vit_status vit_profile_end(vit_model *m, float *total_ms, int32_t *launches);

@@ -30,6 +30,16 @@ vit_status vit_stage_linear(const void *A, const void *W, const float *bias, int
 vit_status vit_stage_attention(const void *qkv, int32_t B, int32_t T, int32_t heads, void *out, int32_t *status,
                                vit_stream_t stream);
 
+/* Position-embedding resize ([diagram] "DINOv2-S encoder": "Bicubic interpolation" of the
+ * learned grid to the input's patch grid), the kernel vit_forward_hw runs first:
+ *   pos: fp32 [(pos_on_cls ? 1 : 0) + gh0 * gw0, D], the patch rows in row-major grid order;
+ *   out: fp32 [(pos_on_cls ? 1 : 0) + gh * gw, D]; the CLS row (if any) is copied, the patch
+ *   rows are the separable cubic-convolution resize (Keys' kernel, a = -0.75, half-pixel
+ *   centres, taps clamped to the border) of the gh0 x gw0 grid to gh x gw.
+ * Grids 1..4096 per side (VIT_E_SHAPE otherwise).  Enqueues on `stream`. */
+vit_status vit_stage_pos_resize(const float *pos, int32_t gh0, int32_t gw0, int32_t gh, int32_t gw, int32_t D,
+                                int32_t pos_on_cls, float *out, vit_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -126,3 +126,15 @@ def test_forward_replays_from_a_cuda_graph():
     assert torch.equal(outs["desc"], eager["desc"]) and torch.equal(outs["patch_tokens"], eager["patch_tokens"])
     del g
     enc.close()
+
+
+@pytest.mark.parametrize("name", ["vitb14_224", "vitg14_224"])
+def test_other_widths(name):
+    """ViT-B/14 and ViT-G/14 widths (DINOv2 blog's model-variant table) through the same kernels."""
+    need_cuda()
+    spec = S.PRESETS[name]
+    w = S.make_weights(spec, 71)
+    im = S.make_images(spec, 2, 72)
+    g = run_gpu(spec, w, im)
+    ref = O.forward(im, w, spec, record_hidden=True)
+    assert_forward_parity(g, ref, spec, [0, 1])

@@ -119,9 +119,15 @@ def test_seg_rejects_bad_arguments():
     im = torch.zeros(3, 320, 480, device="cuda")
     text = torch.zeros(4, spec.dim, device="cuda")
     with pytest.raises(V.VitError) as e:
-        enc.seg(im, text, mode=V.VIT_SEG_WHOLE)          # whole mode needs the native size
-    assert e.value.status == V.VIT_E_UNSUPPORTED
-    with pytest.raises(V.VitError) as e:
         enc.seg(im, text, mode=V.VIT_SEG_SLIDE, side=224, stride=112)   # 8 windows > max_batch 2
     assert e.value.status == V.VIT_E_SHAPE
+    with pytest.raises(V.VitError) as e:
+        enc.seg(im, text, mode=V.VIT_SEG_SLIDE, side=400, stride=112)   # window taller than the image
+    assert e.value.status == V.VIT_E_SHAPE
+    with pytest.raises(V.VitError) as e:
+        enc.seg(im, text, mode=V.VIT_SEG_SLIDE, side=8, stride=112)     # window smaller than a patch
+    assert e.value.status == V.VIT_E_INVALID_ARG
+    with pytest.raises(V.VitError) as e:
+        enc.seg(im, text, mode=7)
+    assert e.value.status == V.VIT_E_INVALID_ARG
     enc.close()

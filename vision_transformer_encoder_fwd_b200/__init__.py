@@ -25,7 +25,7 @@ VIT_E_NONFINITE = 7
 VIT_SEG_WHOLE = 0
 VIT_SEG_SLIDE = 1
 KERNEL_KINDS = ("im2col", "patch_gemm", "prefix", "qkv_gemm", "attention", "proj_gemm", "fc1_gemm", "fc2_gemm",
-                "tap", "final_ln", "seg_norm", "seg_cos", "seg_map")
+                "tap", "final_ln", "seg_norm", "seg_cos", "seg_map", "pos_resize", "head_out")
 
 
 class VitConfig(ctypes.Structure):
@@ -77,6 +77,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "vit_create": (I32, [ctypes.POINTER(VitConfig), ctypes.POINTER(VitWeights), ctypes.POINTER(P)]),
         "vit_workspace_size": (I32, [P, I32, ctypes.POINTER(SZ)]),
         "vit_forward": (I32, [P, P, I32, ctypes.POINTER(VitOutputs), P, SZ, P]),
+        "vit_workspace_size_hw": (I32, [P, I32, I32, I32, ctypes.POINTER(SZ)]),
+        "vit_forward_hw": (I32, [P, P, I32, I32, I32, ctypes.POINTER(VitOutputs), P, SZ, P]),
+        "vit_set_text_head": (I32, [P, ctypes.POINTER(VitBlockWeights), I32]),
+        "vit_forward_text_tokens": (I32, [P, P, I32, I32, I32, P, P, SZ, P]),
         "vit_host_workspace_size": (I32, [P, I32, ctypes.POINTER(SZ)]),
         "vit_forward_host": (I32, [P, P, I32, P, P, P, SZ, P]),
         "vit_forward_noalloc": (I32, [P, P, I32, ctypes.POINTER(VitOutputs), P]),
@@ -91,6 +95,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "vit_profile_end": (I32, [P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(I32)]),
         "vit_stage_linear": (I32, [P, P, P, I32, I32, I32, I32, P, P, P]),
         "vit_stage_attention": (I32, [P, I32, I32, I32, P, P, P]),
+        "vit_stage_pos_resize": (I32, [P, I32, I32, I32, I32, I32, I32, P, P]),
     }
     for name, (res, args) in sigs.items():
         f = getattr(lib, name)
@@ -158,10 +163,19 @@ class VitEncoder:
         self._ws = None
 
     # -------------------------------------------------------------- workspace
-    def workspace_size(self, batch: int) -> int:
+    def workspace_size(self, batch: int, hw=None) -> int:
         n = ctypes.c_size_t()
-        _check("vit_workspace_size", self.lib.vit_workspace_size(self.handle, batch, ctypes.byref(n)))
+        if hw is None or tuple(hw) == (self.spec.img_h, self.spec.img_w):
+            _check("vit_workspace_size", self.lib.vit_workspace_size(self.handle, batch, ctypes.byref(n)))
+        else:
+            _check("vit_workspace_size_hw", self.lib.vit_workspace_size_hw(self.handle, batch, int(hw[0]), int(hw[1]),
+                                                                           ctypes.byref(n)))
         return n.value
+
+    def grid(self, hw=None):
+        """Patch grid (gh, gw) of an H x W input: the stride-p convolution's floor."""
+        H, W = (self.spec.img_h, self.spec.img_w) if hw is None else hw
+        return H // self.spec.patch, W // self.spec.patch
 
     def _workspace(self, nbytes: int):
         import torch
@@ -170,24 +184,27 @@ class VitEncoder:
         return self._ws
 
     # -------------------------------------------------------------- forward
-    def alloc_outputs(self, B: int, desc=True, patch=False, patch_fp32=False, taps=False, hidden=False):
+    def alloc_outputs(self, B: int, desc=True, patch=False, patch_fp32=False, taps=False, hidden=False, hw=None):
         import torch
         s, dev = self.spec, self.device
+        gh, gw = self.grid(hw)
         out = {}
         if desc:
             out["desc"] = torch.empty(B, s.dim, dtype=torch.float32, device=dev)
         if patch:
-            out["patch_tokens"] = torch.empty(B, s.n_patches, s.dim, device=dev,
+            out["patch_tokens"] = torch.empty(B, gh * gw, s.dim, device=dev,
                                               dtype=torch.float32 if patch_fp32 else torch.bfloat16)
         if taps:
-            out["taps"] = [torch.empty(B, s.dim, s.grid_h, s.grid_w, dtype=torch.float32, device=dev) for _ in s.taps]
+            out["taps"] = [torch.empty(B, s.dim, gh, gw, dtype=torch.float32, device=dev) for _ in s.taps]
         if hidden:
-            out["hidden"] = torch.empty(s.depth, B, s.tokens, s.dim, dtype=torch.float32, device=dev)
+            out["hidden"] = torch.empty(s.depth, B, 1 + s.registers + gh * gw, s.dim, dtype=torch.float32, device=dev)
         return out
 
     def forward_into(self, images, outs: Dict[str, object], stream=None, ws=None) -> None:
-        """vit_forward with caller-allocated outputs (see alloc_outputs)."""
-        B = images.shape[0]
+        """vit_forward (vit_forward_hw when images are not img_h x img_w) with caller-allocated
+        outputs (see alloc_outputs)."""
+        B, H, W = images.shape[0], images.shape[-2], images.shape[-1]
+        native = (H, W) == (self.spec.img_h, self.spec.img_w)
         o = VitOutputs()
         o.desc = _ptr(outs.get("desc"))
         pt = outs.get("patch_tokens")
@@ -196,13 +213,18 @@ class VitEncoder:
         for i, t in enumerate(outs.get("taps", [])[:4]):
             o.taps[i] = _ptr(t)
         o.hidden = _ptr(outs.get("hidden"))
-        need = self.workspace_size(B)
+        need = self.workspace_size(B, (H, W))
         wsb = ws if ws is not None else self._workspace(need)
-        _check("vit_forward", self.lib.vit_forward(self.handle, _ptr(images), B, ctypes.byref(o), _ptr(wsb),
-                                                   wsb.numel(), _stream_handle(stream)))
+        if native:
+            _check("vit_forward", self.lib.vit_forward(self.handle, _ptr(images), B, ctypes.byref(o), _ptr(wsb),
+                                                       wsb.numel(), _stream_handle(stream)))
+        else:
+            _check("vit_forward_hw", self.lib.vit_forward_hw(self.handle, _ptr(images), B, H, W, ctypes.byref(o),
+                                                             _ptr(wsb), wsb.numel(), _stream_handle(stream)))
 
     def forward(self, images, desc=True, patch=False, patch_fp32=False, taps=False, hidden=False, stream=None):
-        outs = self.alloc_outputs(images.shape[0], desc, patch, patch_fp32, taps, hidden)
+        outs = self.alloc_outputs(images.shape[0], desc, patch, patch_fp32, taps, hidden,
+                                  hw=(images.shape[-2], images.shape[-1]))
         self.forward_into(images, outs, stream)
         return outs
 
@@ -219,6 +241,32 @@ class VitEncoder:
         _check("vit_forward_host", self.lib.vit_forward_host(
             self.handle, _ptr(images_host), B, _ptr(desc_host), _ptr(patch_host), _ptr(wsb), wsb.numel(),
             _stream_handle(stream)))
+
+    # -------------------------------------------------------------- dino.txt vision head
+    def set_text_head(self, head_blocks) -> None:
+        """vit_set_text_head: attach the dino.txt vision head (list of per-block bf16 weight dicts)."""
+        import torch
+        self.head_w = [{k: v.to(device=self.device, dtype=torch.bfloat16).contiguous() for k, v in b.items()}
+                       for b in head_blocks]
+        arr = (VitBlockWeights * len(self.head_w))()
+        for i, b in enumerate(self.head_w):
+            for n in _BLOCK_FIELDS:
+                setattr(arr[i], n, _ptr(b[n]))
+        self._head_arr = arr
+        with torch.cuda.device(self.device):
+            _check("vit_set_text_head", self.lib.vit_set_text_head(self.handle, arr, len(self.head_w)))
+
+    def text_tokens(self, images, stream=None):
+        """vit_forward_text_tokens: backbone + head -> fp32 patch tokens [B, gh*gw, D]."""
+        import torch
+        B, H, W = images.shape[0], images.shape[-2], images.shape[-1]
+        gh, gw = self.grid((H, W))
+        tok = torch.empty(B, gh * gw, self.spec.dim, dtype=torch.float32, device=self.device)
+        need = self.workspace_size(B, (H, W))
+        wsb = self._workspace(need)
+        _check("vit_forward_text_tokens", self.lib.vit_forward_text_tokens(
+            self.handle, _ptr(images), B, H, W, _ptr(tok), _ptr(wsb), wsb.numel(), _stream_handle(stream)))
+        return tok
 
     # -------------------------------------------------------------- zero-shot
     def seg_workspace_size(self, H, W, C, mode, side, stride) -> int:
@@ -295,3 +343,14 @@ def stage_attention(qkv, heads: int, out=None, status=None, stream=None):
     _check("vit_stage_attention", lib.vit_stage_attention(_ptr(qkv), B, T, heads, _ptr(out), _ptr(st),
                                                           _stream_handle(stream)))
     return out, st
+
+
+def stage_pos_resize(pos, grid0, grid, pos_on_cls: bool, stream=None):
+    """vit_stage_pos_resize: fp32 pos [(cls) + gh0*gw0, D] -> [(cls) + gh*gw, D] on the device."""
+    import torch
+    lib = load_library()
+    D = pos.shape[1]
+    out = torch.empty((1 if pos_on_cls else 0) + grid[0] * grid[1], D, dtype=torch.float32, device=pos.device)
+    _check("vit_stage_pos_resize", lib.vit_stage_pos_resize(_ptr(pos), grid0[0], grid0[1], grid[0], grid[1], D,
+                                                            1 if pos_on_cls else 0, _ptr(out), _stream_handle(stream)))
+    return out

@@ -93,6 +93,59 @@ __global__ void prefix_tokens_kernel(const float* __restrict__ cls, const float*
   if (lane == 0) stats[row * (D / gcols) + g] = make_float2(mean, q);
 }
 
+// [diagram] "DINOv2-S encoder": the learned position grid goes through "Bicubic
+// interpolation" to the input's patch grid.  Separable cubic convolution with Keys' kernel
+// (a = -0.75), half-pixel centres (source coordinate (i + 1/2) * in/out - 1/2, not clamped),
+// the four taps of each axis clamped to the border; a CLS row (pos_off = 1) is copied as is.
+// One thread per output element, D innermost: a warp reads 32 consecutive floats of each of
+// the 16 source rows it touches.
+__device__ __forceinline__ void keys_cubic_weights(float t, float w[4]) {
+  const float a = -0.75f;
+  // |x| <= 1: ((a + 2)|x| - (a + 3)) x^2 + 1;   1 < |x| < 2: a|x|^3 - 5a x^2 + 8a|x| - 4a
+  auto near = [a](float x) { return ((a + 2.f) * x - (a + 3.f)) * x * x + 1.f; };
+  auto far = [a](float x) { return ((a * x - 5.f * a) * x + 8.f * a) * x - 4.f * a; };
+  w[0] = far(1.f + t);
+  w[1] = near(t);
+  w[2] = near(1.f - t);
+  w[3] = far(2.f - t);
+}
+
+__global__ void pos_resize_kernel(const float* __restrict__ pos0, int gh0, int gw0, int gh, int gw, int D, int pos_off,
+                                  float* __restrict__ out) {
+  const long long total = static_cast<long long>(pos_off + gh * gw) * D;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int d = static_cast<int>(i % D);
+    const int r = static_cast<int>(i / D);
+    if (r < pos_off) {
+      out[i] = pos0[i];
+      continue;
+    }
+    const int pi = r - pos_off, py = pi / gw, px = pi - py * gw;
+    const float sy = (static_cast<float>(py) + 0.5f) * (static_cast<float>(gh0) / static_cast<float>(gh)) - 0.5f;
+    const float sx = (static_cast<float>(px) + 0.5f) * (static_cast<float>(gw0) / static_cast<float>(gw)) - 0.5f;
+    const float fy = floorf(sy), fx = floorf(sx);
+    float wy[4], wx[4];
+    keys_cubic_weights(sy - fy, wy);
+    keys_cubic_weights(sx - fx, wx);
+    const int iy = static_cast<int>(fy) - 1, ix = static_cast<int>(fx) - 1;
+    const float* base = pos0 + static_cast<size_t>(pos_off) * D + d;
+    float acc = 0.f;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int yy = min(max(iy + a, 0), gh0 - 1);
+      float rowv = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int xx = min(max(ix + c, 0), gw0 - 1);
+        rowv = fmaf(wx[c], base[static_cast<size_t>(yy * gw0 + xx) * D], rowv);
+      }
+      acc = fmaf(wy[a], rowv, acc);
+    }
+    out[i] = acc;
+  }
+}
+
 // Row LayerNorm statistics with one warp per row, two passes over the row (L1/L2-resident on
 // the second pass): biased variance, eps inside the square root ([diagram] "Encoder block").
 __device__ __forceinline__ void row_mean_rstd(const float* __restrict__ xr, int D, float eps, float& mean, float& rstd) {
@@ -148,6 +201,69 @@ __global__ void final_ln_kernel(const float* __restrict__ x, const float* __rest
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(patch) + o;
       for (int n = lane; n < D; n += 32) dst[n] = __float2bfloat16_rn((xr[n] - mean) * rstd * g[n] + be[n]);
     }
+  }
+}
+
+// [dino.txt article] the vision head's 2 blocks run on the backbone's final-norm sequence: the
+// final LayerNorm applied in place to every row of the residual stream x (CLS, registers and
+// patches), with the bf16 copy xb and the per-group (mean, M2) statistics that the first head
+// block's folded LN1 reads -- the state a backbone block leaves behind.  One warp per row; each
+// group of gcols (64 or 128) columns is kept in registers between its two passes.
+__global__ void final_ln_stream_kernel(float* __restrict__ x, const float* __restrict__ g,
+                                       const float* __restrict__ be, long long rows, int D, float eps, int gcols,
+                                       __nv_bfloat16* __restrict__ xb, float2* __restrict__ stats) {
+  const int warps_per_block = blockDim.x >> 5;
+  const long long row = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int lane = threadIdx.x & 31;
+  float* xr = x + static_cast<size_t>(row) * D;
+  float mean, rstd;
+  row_mean_rstd(xr, D, eps, mean, rstd);
+  __syncwarp();
+  const int per = gcols / 32;  // 2 or 4
+  const int ng = D / gcols;
+  for (int gi = 0; gi < ng; ++gi) {
+    float v[4];
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (j < per) {
+        const int n = gi * gcols + j * 32 + lane;
+        v[j] = (xr[n] - mean) * rstd * g[n] + be[n];
+        s += v[j];
+      }
+    }
+    const float gm = warp_sum(s) / static_cast<float>(gcols);
+    float q = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (j < per) {
+        const int n = gi * gcols + j * 32 + lane;
+        const float d = v[j] - gm;
+        q = fmaf(d, d, q);
+        xr[n] = v[j];
+        xb[static_cast<size_t>(row) * D + n] = __float2bfloat16_rn(v[j]);
+      }
+    }
+    q = warp_sum(q);
+    if (lane == 0) stats[static_cast<size_t>(row) * ng + gi] = make_float2(gm, q);
+  }
+}
+
+// The patch rows of the residual stream, fp32: tok[b, p, :] = x[b, 1 + R + p, :] (the dino.txt
+// head's output tokens, CLS and registers dropped).  float4 copies, grid-stride.
+__global__ void patch_rows_kernel(const float* __restrict__ x, int B, int T, int R, int D, float* __restrict__ tok) {
+  const int P = T - 1 - R;
+  const int d4 = D / 4;
+  const long long total = static_cast<long long>(B) * P * d4;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(i % d4);
+    const long long r = i / d4;
+    const int b = static_cast<int>(r / P);
+    const int p = static_cast<int>(r - static_cast<long long>(b) * P);
+    reinterpret_cast<float4*>(tok)[i] =
+        reinterpret_cast<const float4*>(x + (static_cast<size_t>(b) * T + 1 + R + p) * D)[c];
   }
 }
 

@@ -11,9 +11,10 @@
 //                      the epilogue.
 //   warps 2..9         epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, i.e. one output
 //                      row per thread, and half of the tile's columns (warps 2..5 the first
-//                      half, 6..9 the second), 32 columns per tcgen05.ld; applies the epilogue
-//                      and writes global memory, then releases the accumulator.  Two warps per
-//                      lane quarter give each SM sub-partition two epilogue warps to overlap.
+//                      half, 6..9 the second), 32 columns per tcgen05.ld.  Results are packed
+//                      into a swizzled per-warp staging buffer in shared memory and written by
+//                      TMA stores (the residual stream x is also read by TMA, one chunk ahead),
+//                      so global memory only sees whole 128-byte lines.
 // The double-buffered accumulator lets the epilogue of tile i overlap the MMAs of tile i+1.
 #pragma once
 
@@ -24,7 +25,8 @@ namespace vit {
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 64;
 constexpr int GEMM_THREADS = 320;
-constexpr int GEMM_EPI_THREADS = 256;
+constexpr int GEMM_EPI_WARPS = 8;
+constexpr int GEMM_EPI_THREADS = 32 * GEMM_EPI_WARPS;
 
 enum EpiMode : int {
   EPI_BIAS = 0,    // out_bf16 = act(acc + bias)
@@ -37,7 +39,6 @@ struct EpiParams {
   int M, N;
   const float* bias;  // [N]
   int gelu;           // BIAS / LNFOLD: apply exact-erf GELU
-  __nv_bfloat16* out;  // BIAS / LNFOLD output [M, ldo]
   int ldo;
   // LNFOLD: per-row LayerNorm statistics rebuilt from partials written by the producer of x
   const float* colsum;     // [N] column sums of the gamma-folded weight
@@ -45,7 +46,7 @@ struct EpiParams {
   int nt, nt_cols, D;
   float eps;
   // RESID / PATCH
-  float* x;              // [rows, N] fp32 residual stream
+  float* x;              // [rows, N] fp32 residual stream (PATCH writes it directly)
   __nv_bfloat16* xb;     // [rows, N] bf16 copy of x (A operand of the next folded GEMM)
   const float* ls;       // [N] layer scale (RESID)
   float2* stats_out;     // [rows, N / (BN/2)] (mean, M2) over each group of BN/2 columns
@@ -54,15 +55,22 @@ struct EpiParams {
   int P, T, R, pos_off;
 };
 
-template <int BN>
+template <int BN, int MODE>
 struct GemmCfg {
-  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int STAGES = (MODE == EPI_RESID) ? 3 : ((BN == 256) ? 4 : 6);
   static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
   static constexpr int B_BYTES = BN * GEMM_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+  // per epilogue warp: RESID two 32 x 32 fp32 x buffers (128-byte rows, 128B swizzle) and one
+  // 32 x 32 bf16 buffer (64-byte rows, 64B swizzle); BIAS / LNFOLD one 32 x 64 bf16 buffer
+  static constexpr int EPI_WARP_BYTES = (MODE == EPI_RESID) ? (2 * 4096 + 2048) : (MODE == EPI_PATCH ? 0 : 4096);
+  static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
+  static constexpr int OFF_BAR = OFF_EPI + GEMM_EPI_WARPS * EPI_WARP_BYTES;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(8 * (2 * STAGES + 5 + 2 * GEMM_EPI_WARPS) + 8 <= BAR_BYTES, "barrier area");
 };
 
 __device__ __forceinline__ void merge_stats(float& n, float& mean, float& m2, float nb, float mb, float m2b) {
@@ -73,17 +81,48 @@ __device__ __forceinline__ void merge_stats(float& n, float& mean, float& m2, fl
   n = tot;
 }
 
-// One thread's part of a tile: row `row`, columns n0 .. n0 + BN/2 - 1 (TMEM columns from taddr).
-// RESID: `xpre` holds the first 32 columns of x for this row, loaded before the accumulator was
-// ready; each following chunk of x is loaded while the current one is being processed.
+// Affine epilogue of one 32-column chunk for BIAS / LNFOLD: v <- act(rstd * v - rstd * mu * c + b).
+template <int MODE>
+__device__ __forceinline__ void epi_affine(const EpiParams& ep, float (&v)[32], int n, float mu, float rstd) {
+  const float4* b4 = reinterpret_cast<const float4*>(ep.bias + n);
+  if (MODE == EPI_LNFOLD) {
+    const float4* c4 = reinterpret_cast<const float4*>(ep.colsum + n);
+    const float rm = rstd * mu;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 bb = __ldg(b4 + j);
+      const float4 cc = __ldg(c4 + j);
+      v[4 * j + 0] = fmaf(rstd, v[4 * j + 0], fmaf(-rm, cc.x, bb.x));
+      v[4 * j + 1] = fmaf(rstd, v[4 * j + 1], fmaf(-rm, cc.y, bb.y));
+      v[4 * j + 2] = fmaf(rstd, v[4 * j + 2], fmaf(-rm, cc.z, bb.z));
+      v[4 * j + 3] = fmaf(rstd, v[4 * j + 3], fmaf(-rm, cc.w, bb.w));
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 bb = __ldg(b4 + j);
+      v[4 * j + 0] += bb.x;
+      v[4 * j + 1] += bb.y;
+      v[4 * j + 2] += bb.z;
+      v[4 * j + 3] += bb.w;
+    }
+  }
+  if (ep.gelu) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+  }
+}
+
+// BIAS / LNFOLD: one warp's half of a tile (rows row0 .. row0 + 31, columns n0 .. n0 + BN/2 - 1),
+// 64 columns per TMA store from the warp's staging buffer `obuf` (32 rows x 128 bytes, 128B
+// swizzle: 16-byte chunk k of row r sits at chunk k ^ (r % 8)).
 template <int BN, int MODE>
-__device__ __forceinline__ void gemm_epilogue_tile(const EpiParams& ep, uint32_t taddr, int row, int n0,
-                                                   float4 (&xpre)[8]) {
-  constexpr int HALF = BN / 2;
-  constexpr int CHUNKS = HALF / 32;
-  const bool valid = row < ep.M;
+__device__ __forceinline__ void epilogue_store_bf16(const EpiParams& ep, const CUtensorMap* tmO, uint32_t taddr,
+                                                    int row0, int n0, uint8_t* obuf) {
+  const int lane = threadIdx.x & 31;
+  const int row = row0 + lane;
   float mu = 0.f, rstd = 0.f;
-  if (MODE == EPI_LNFOLD && valid) {
+  if (MODE == EPI_LNFOLD && row < ep.M) {
     float n = 0.f, mean = 0.f, m2 = 0.f;
     const float2* s = ep.stats_in + static_cast<size_t>(row) * ep.nt;
     for (int t = 0; t < ep.nt; ++t) {
@@ -93,145 +132,201 @@ __device__ __forceinline__ void gemm_epilogue_tile(const EpiParams& ep, uint32_t
     mu = mean;
     rstd = rsqrtf(m2 / static_cast<float>(ep.D) + ep.eps);
   }
+#pragma unroll 1
+  for (int g = 0; g < BN / 128; ++g) {
+    if (lane == 0) tma_store_wait_read0();  // the previous store has left the staging buffer
+    __syncwarp();
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int c = 2 * g + cc;
+      float v[32];
+      tmem_ld32(taddr + c * 32, v);
+      epi_affine<MODE>(ep, v, n0 + c * 32, mu, rstd);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * k + 0], v[8 * k + 1]);
+        w.y = pack_bf16x2(v[8 * k + 2], v[8 * k + 3]);
+        w.z = pack_bf16x2(v[8 * k + 4], v[8 * k + 5]);
+        w.w = pack_bf16x2(v[8 * k + 6], v[8 * k + 7]);
+        const int chunk = (cc * 4 + k) ^ (lane & 7);
+        *reinterpret_cast<uint4*>(obuf + lane * 128 + chunk * 16) = w;
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmO, obuf, n0 + g * 64, row0);
+      tma_store_commit();
+    }
+  }
+}
+
+// RESID: one warp's half of a tile.  x arrives by TMA into xbuf[c & 1] (32 rows x 128 bytes, 128B
+// swizzle), chunk c + 1 is requested while chunk c is processed; the updated x goes back into the
+// same buffer and, with its bf16 copy (xbbuf: 32 rows x 64 bytes, 64B swizzle), out by TMA stores.
+// Row statistics (mean, M2) of the warp's BN/2 columns are written per row.
+template <int BN>
+__device__ __forceinline__ void epilogue_resid(const EpiParams& ep, const CUtensorMap* tmX, const CUtensorMap* tmXb,
+                                               uint32_t taddr, int row0, int n0, uint8_t* xbuf0, uint8_t* xbbuf,
+                                               uint64_t* xfull, uint32_t (&xph)[2], bool (&xpending)[2],
+                                               volatile int* abort_flag, int* gstatus, bool& ok) {
+  constexpr int HALF = BN / 2;
+  constexpr int CHUNKS = HALF / 32;
+  const int lane = threadIdx.x & 31;
+  const int row = row0 + lane;
+  float run_n = 0.f, run_mean = 0.f, run_m2 = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < CHUNKS; ++c) {
+    const int buf = c & 1;
+    const int n = n0 + c * 32;
+    if (lane == 0) {
+      tma_store_wait_read0();  // earlier stores have left xbuf[buf ^ 1] and xbbuf
+      if (c + 1 < CHUNKS) {
+        mbar_arrive_expect_tx(&xfull[buf ^ 1], 4096);
+        tma_load_2d(xbuf0 + (buf ^ 1) * 4096, tmX, n + 32, row0, &xfull[buf ^ 1]);
+        xpending[buf ^ 1] = true;
+      }
+    }
+    __syncwarp();
+    if (!mbar_wait(&xfull[buf], xph[buf], abort_flag, gstatus, DEV_TIMEOUT_GEMM + 6)) {
+      ok = false;
+      return;
+    }
+    xph[buf] ^= 1u;
+    if (lane == 0) xpending[buf] = false;
+    float v[32];
+    __syncwarp();
+    tmem_ld32(taddr + c * 32, v);
+    uint8_t* xr = xbuf0 + buf * 4096 + lane * 128;
+    const float4* b4 = reinterpret_cast<const float4*>(ep.bias + n);
+    const float4* l4 = reinterpret_cast<const float4*>(ep.ls + n);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float4* xp = reinterpret_cast<float4*>(xr + ((k ^ (lane & 7)) << 4));
+      const float4 xo = *xp;
+      const float4 bb = __ldg(b4 + k);
+      const float4 ll = __ldg(l4 + k);
+      v[4 * k + 0] = fmaf(ll.x, v[4 * k + 0] + bb.x, xo.x);
+      v[4 * k + 1] = fmaf(ll.y, v[4 * k + 1] + bb.y, xo.y);
+      v[4 * k + 2] = fmaf(ll.z, v[4 * k + 2] + bb.z, xo.z);
+      v[4 * k + 3] = fmaf(ll.w, v[4 * k + 3] + bb.w, xo.w);
+      *xp = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint4 w;
+      w.x = pack_bf16x2(v[8 * k + 0], v[8 * k + 1]);
+      w.y = pack_bf16x2(v[8 * k + 2], v[8 * k + 3]);
+      w.z = pack_bf16x2(v[8 * k + 4], v[8 * k + 5]);
+      w.w = pack_bf16x2(v[8 * k + 6], v[8 * k + 7]);
+      *reinterpret_cast<uint4*>(xbbuf + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) = w;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmX, xbuf0 + buf * 4096, n, row0);
+      tma_store_2d(tmXb, xbbuf, n, row0);
+      tma_store_commit();
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) s += v[j];
+    const float cm = s * (1.0f / 32.0f);
+    float q = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float d = v[j] - cm;
+      q = fmaf(d, d, q);
+    }
+    merge_stats(run_n, run_mean, run_m2, 32.f, cm, q);
+  }
+  if (row < ep.M) ep.stats_out[static_cast<size_t>(row) * (ep.N / HALF) + n0 / HALF] = make_float2(run_mean, run_m2);
+}
+
+// PATCH: rows of the GEMM are scattered to token rows, so this epilogue writes directly.
+template <int BN>
+__device__ __forceinline__ void epilogue_patch(const EpiParams& ep, uint32_t taddr, int row, int n0) {
+  constexpr int HALF = BN / 2;
+  const bool valid = row < ep.M;
   int xrow = row;
   const float* posrow = nullptr;
-  if (MODE == EPI_PATCH && valid) {
+  if (valid) {
     const int b = row / ep.P;
     const int p = row - b * ep.P;
     xrow = b * ep.T + 1 + ep.R + p;
     posrow = ep.pos + static_cast<size_t>(p + ep.pos_off) * ep.N;
   }
   float run_n = 0.f, run_mean = 0.f, run_m2 = 0.f;
-
 #pragma unroll 1
-  for (int c = 0; c < CHUNKS; ++c) {
+  for (int c = 0; c < HALF / 32; ++c) {
     float v[32];
     const int n = n0 + c * 32;
-    float4 xc[8];
-    if (MODE == EPI_RESID) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) xc[j] = xpre[j];
-      if (valid && c + 1 < CHUNKS) {
-        const float4* xn = reinterpret_cast<const float4*>(ep.x + static_cast<size_t>(xrow) * ep.N + n + 32);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) xpre[j] = xn[j];
-      }
-    }
     __syncwarp();
     tmem_ld32(taddr + c * 32, v);
     if (valid) {
-      if (MODE == EPI_BIAS || MODE == EPI_LNFOLD) {
-        const float4* b4 = reinterpret_cast<const float4*>(ep.bias + n);
-        if (MODE == EPI_LNFOLD) {
-          const float4* c4 = reinterpret_cast<const float4*>(ep.colsum + n);
-          const float rm = rstd * mu;
+      const float4* b4 = reinterpret_cast<const float4*>(ep.bias + n);
+      const float4* p4 = reinterpret_cast<const float4*>(posrow + n);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 bb = __ldg(b4 + j);
-            const float4 cc = __ldg(c4 + j);
-            v[4 * j + 0] = fmaf(rstd, v[4 * j + 0], fmaf(-rm, cc.x, bb.x));
-            v[4 * j + 1] = fmaf(rstd, v[4 * j + 1], fmaf(-rm, cc.y, bb.y));
-            v[4 * j + 2] = fmaf(rstd, v[4 * j + 2], fmaf(-rm, cc.z, bb.z));
-            v[4 * j + 3] = fmaf(rstd, v[4 * j + 3], fmaf(-rm, cc.w, bb.w));
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 bb = __ldg(b4 + j);
-            v[4 * j + 0] += bb.x;
-            v[4 * j + 1] += bb.y;
-            v[4 * j + 2] += bb.z;
-            v[4 * j + 3] += bb.w;
-          }
-        }
-        if (ep.gelu) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
-        }
-        uint4* o = reinterpret_cast<uint4*>(ep.out + static_cast<size_t>(row) * ep.ldo + n);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 w;
-          w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-          w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-          w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-          w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-          o[j] = w;
-        }
-      } else {
-        float4* xp = reinterpret_cast<float4*>(ep.x + static_cast<size_t>(xrow) * ep.N + n);
-        const float4* b4 = reinterpret_cast<const float4*>(ep.bias + n);
-        if (MODE == EPI_RESID) {
-          const float4* l4 = reinterpret_cast<const float4*>(ep.ls + n);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 xo = xc[j];
-            const float4 bb = __ldg(b4 + j);
-            const float4 ll = __ldg(l4 + j);
-            v[4 * j + 0] = fmaf(ll.x, v[4 * j + 0] + bb.x, xo.x);
-            v[4 * j + 1] = fmaf(ll.y, v[4 * j + 1] + bb.y, xo.y);
-            v[4 * j + 2] = fmaf(ll.z, v[4 * j + 2] + bb.z, xo.z);
-            v[4 * j + 3] = fmaf(ll.w, v[4 * j + 3] + bb.w, xo.w);
-          }
-        } else {
-          const float4* p4 = reinterpret_cast<const float4*>(posrow + n);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 bb = __ldg(b4 + j);
-            const float4 pp = __ldg(p4 + j);
-            v[4 * j + 0] += bb.x + pp.x;
-            v[4 * j + 1] += bb.y + pp.y;
-            v[4 * j + 2] += bb.z + pp.z;
-            v[4 * j + 3] += bb.w + pp.w;
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) xp[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-        uint4* o = reinterpret_cast<uint4*>(ep.xb + static_cast<size_t>(xrow) * ep.N + n);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 w;
-          w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-          w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-          w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-          w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-          o[j] = w;
-        }
-        float s = 0.f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) s += v[j];
-        const float cm = s * (1.0f / 32.0f);
-        float q = 0.f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float d = v[j] - cm;
-          q = fmaf(d, d, q);
-        }
-        merge_stats(run_n, run_mean, run_m2, 32.f, cm, q);
+      for (int j = 0; j < 8; ++j) {
+        const float4 bb = __ldg(b4 + j);
+        const float4 pp = __ldg(p4 + j);
+        v[4 * j + 0] += bb.x + pp.x;
+        v[4 * j + 1] += bb.y + pp.y;
+        v[4 * j + 2] += bb.z + pp.z;
+        v[4 * j + 3] += bb.w + pp.w;
       }
+      float4* xp = reinterpret_cast<float4*>(ep.x + static_cast<size_t>(xrow) * ep.N + n);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xp[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      uint4* o = reinterpret_cast<uint4*>(ep.xb + static_cast<size_t>(xrow) * ep.N + n);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+        w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+        w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+        w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+        o[j] = w;
+      }
+      float s = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) s += v[j];
+      const float cm = s * (1.0f / 32.0f);
+      float q = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float d = v[j] - cm;
+        q = fmaf(d, d, q);
+      }
+      merge_stats(run_n, run_mean, run_m2, 32.f, cm, q);
     }
   }
-  if ((MODE == EPI_RESID || MODE == EPI_PATCH) && valid) {
-    ep.stats_out[static_cast<size_t>(xrow) * (ep.N / HALF) + n0 / HALF] = make_float2(run_mean, run_m2);
-  }
+  if (valid) ep.stats_out[static_cast<size_t>(xrow) * (ep.N / HALF) + n0 / HALF] = make_float2(run_mean, run_m2);
 }
 
+// tmO1 / tmO2: BIAS / LNFOLD -> tmO1 = output [M, ldo] bf16 (box 64 x 32, 128B swizzle);
+//              RESID -> tmO1 = x [M, N] fp32 (box 32 x 32, 128B swizzle), tmO2 = xb [M, N] bf16
+//              (box 32 x 32, 64B swizzle); PATCH -> unused.
 template <int BN, int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
-    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
+    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmO1, const __grid_constant__ CUtensorMap tmO2, int M,
                         int N, int K, EpiParams ep, int* gstatus) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, MODE>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint8_t* sEpi = smem + Cfg::OFF_EPI;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* xfull = mma_done + 1;  // [GEMM_EPI_WARPS][2] (RESID)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(xfull + 2 * GEMM_EPI_WARPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -248,9 +343,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(&tempty[a], GEMM_EPI_THREADS);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < 2 * GEMM_EPI_WARPS; ++i) mbar_init(&xfull[i], 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (MODE != EPI_PATCH) tma_prefetch_desc(&tmO1);
+    if (MODE == EPI_RESID) tma_prefetch_desc(&tmO2);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, Cfg::TMEM_COLS);
@@ -341,35 +439,56 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     __syncwarp();
   } else if (!skip && warp >= 2) {
     // ---------------------------------------------------------------- epilogue
+    const int e = warp - 2;
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int half = e >> 2;
+    uint8_t* wbuf = sEpi + e * Cfg::EPI_WARP_BYTES;
+    uint64_t* wxfull = xfull + 2 * e;
+    uint32_t xph[2] = {0u, 0u};
+    bool xpending[2] = {false, false};
+    bool ok = true;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       const int mb = tile / num_n;
       const int nb = tile - mb * num_n;
-      float4 xpre[8];
-      if (MODE == EPI_RESID) {
-        // this thread's first 32 columns of x, loaded while the accumulator is still being built
-        const int row0 = mb * GEMM_BM + q * 32 + lane;
-        if (row0 < M) {
-          const float4* xs = reinterpret_cast<const float4*>(ep.x + static_cast<size_t>(row0) * ep.N + nb * BN +
-                                                             half * (BN / 2));
-#pragma unroll
-          for (int j = 0; j < 8; ++j) xpre[j] = xs[j];
-        }
+      const int row0 = mb * GEMM_BM + q * 32;
+      const int n0 = nb * BN + half * (BN / 2);
+      if (MODE == EPI_RESID && lane == 0) {
+        // the tile's first chunk of x, requested before the accumulator is ready
+        tma_store_wait_read0();
+        mbar_arrive_expect_tx(&wxfull[0], 4096);
+        tma_load_2d(wbuf, &tmO1, n0, row0, &wxfull[0]);
+        xpending[0] = true;
       }
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 4)) break;
       tc_fence_after();
-      const int row = mb * GEMM_BM + q * 32 + lane;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + half * (BN / 2));
-      gemm_epilogue_tile<BN, MODE>(ep, taddr, row, nb * BN + half * (BN / 2), xpre);
+      __syncwarp();
+      if (MODE == EPI_RESID) {
+        epilogue_resid<BN>(ep, &tmO1, &tmO2, taddr, row0, n0, wbuf, wbuf + 8192, wxfull, xph, xpending, abort_flag,
+                           gstatus, ok);
+        if (!ok) break;
+      } else if (MODE == EPI_PATCH) {
+        epilogue_patch<BN>(ep, taddr, row0 + lane, n0);
+      } else {
+        epilogue_store_bf16<BN, MODE>(ep, &tmO1, taddr, row0, n0, wbuf);
+      }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (lane == 0) {
+      if (MODE == EPI_RESID) {
+        // x loads requested but not consumed (only after an abort) must land before exit
+        for (int bb = 0; bb < 2; ++bb)
+          if (xpending[bb]) mbar_wait_drain(&wxfull[bb], xph[bb]);
+      }
+      tma_store_wait0();  // every TMA store of this warp has completed
+    }
+    __syncwarp();
   }
 
   // ---------------------------------------------------------------- teardown

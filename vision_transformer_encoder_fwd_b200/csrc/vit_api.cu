@@ -105,6 +105,40 @@ bool tmap_2d(CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows, ui
   return true;
 }
 
+// 2-D map of an arbitrary element type for the epilogue's TMA stores and x loads: row-major
+// [rows, cols] with leading dimension ld (elements), box box_cols x box_rows, given swizzle.
+bool tmap_2d_any(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype, uint32_t elem_bytes, uint64_t cols,
+                 uint64_t rows, uint64_t ld, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    set_err("cuTensorMapEncodeTiled is not available from the driver");
+    return false;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * elem_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(tm, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_err("cuTensorMapEncodeTiled(epilogue map) failed with %d", static_cast<int>(r));
+    return false;
+  }
+  return true;
+}
+// bf16 output [M, ld] stored in boxes of 64 columns x 32 rows (one epilogue warp, 128B swizzle)
+bool tmap_out_bf16(CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows, uint64_t ld) {
+  return tmap_2d_any(tm, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cols, rows, ld, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// fp32 residual stream [M, D] in boxes of 32 columns x 32 rows (128B swizzle)
+bool tmap_x_f32(CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows) {
+  return tmap_2d_any(tm, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, cols, rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// bf16 copy of x [M, D] in boxes of 32 columns x 32 rows (64B swizzle)
+bool tmap_xb_bf16(CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows) {
+  return tmap_2d_any(tm, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cols, rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 // 3-D bf16 map over qkv [B, T, 3D]: dims {3D, T, B}, box {64, 128, 1}.
 bool tmap_qkv3d(CUtensorMap* tm, const void* base, int B, int T, int D) {
   EncodeTiledFn fn = encode_fn();
@@ -145,32 +179,36 @@ cudaError_t set_smem_attr_once(K kernel, int bytes, std::atomic<uint64_t>& done)
 }
 
 template <int BN, int MODE>
-cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, const EpiParams& ep,
-                          int* st, cudaStream_t s, int nsm) {
+cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o1, const CUtensorMap& o2,
+                          int M, int N, int K, const EpiParams& ep, int* st, cudaStream_t s, int nsm) {
   static std::atomic<uint64_t> attr_done{0};
-  cudaError_t e = set_smem_attr_once(gemm_bf16_tc_kernel<BN, MODE>, GemmCfg<BN>::SMEM_BYTES, attr_done);
+  constexpr int smem = GemmCfg<BN, MODE>::SMEM_BYTES;
+  cudaError_t e = set_smem_attr_once(gemm_bf16_tc_kernel<BN, MODE>, smem, attr_done);
   if (e != cudaSuccess) return e;
   const int tiles = ((M + GEMM_BM - 1) / GEMM_BM) * (N / BN);
   const int grid = std::max(1, std::min(tiles, nsm));
-  gemm_bf16_tc_kernel<BN, MODE><<<grid, GEMM_THREADS, GemmCfg<BN>::SMEM_BYTES, s>>>(a, b, M, N, K, ep, st);
+  gemm_bf16_tc_kernel<BN, MODE><<<grid, GEMM_THREADS, smem, s>>>(a, b, o1, o2, M, N, K, ep, st);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(int bn, int mode, const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
-                        const EpiParams& ep, int* st, cudaStream_t s, int nsm) {
+// o1 / o2: BIAS, LNFOLD: o1 = bf16 output map (tmap_out_bf16); RESID: o1 = x (tmap_x_f32),
+// o2 = xb (tmap_xb_bf16); PATCH: not read (any valid map).
+cudaError_t launch_gemm(int bn, int mode, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o1,
+                        const CUtensorMap& o2, int M, int N, int K, const EpiParams& ep, int* st, cudaStream_t s,
+                        int nsm) {
   if (bn == 256) {
     switch (mode) {
-      case EPI_BIAS: return launch_gemm_t<256, EPI_BIAS>(a, b, M, N, K, ep, st, s, nsm);
-      case EPI_LNFOLD: return launch_gemm_t<256, EPI_LNFOLD>(a, b, M, N, K, ep, st, s, nsm);
-      case EPI_RESID: return launch_gemm_t<256, EPI_RESID>(a, b, M, N, K, ep, st, s, nsm);
-      default: return launch_gemm_t<256, EPI_PATCH>(a, b, M, N, K, ep, st, s, nsm);
+      case EPI_BIAS: return launch_gemm_t<256, EPI_BIAS>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
+      case EPI_LNFOLD: return launch_gemm_t<256, EPI_LNFOLD>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
+      case EPI_RESID: return launch_gemm_t<256, EPI_RESID>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
+      default: return launch_gemm_t<256, EPI_PATCH>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
     }
   }
   switch (mode) {
-    case EPI_BIAS: return launch_gemm_t<128, EPI_BIAS>(a, b, M, N, K, ep, st, s, nsm);
-    case EPI_LNFOLD: return launch_gemm_t<128, EPI_LNFOLD>(a, b, M, N, K, ep, st, s, nsm);
-    case EPI_RESID: return launch_gemm_t<128, EPI_RESID>(a, b, M, N, K, ep, st, s, nsm);
-    default: return launch_gemm_t<128, EPI_PATCH>(a, b, M, N, K, ep, st, s, nsm);
+    case EPI_BIAS: return launch_gemm_t<128, EPI_BIAS>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
+    case EPI_LNFOLD: return launch_gemm_t<128, EPI_LNFOLD>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
+    case EPI_RESID: return launch_gemm_t<128, EPI_RESID>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
+    default: return launch_gemm_t<128, EPI_PATCH>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
   }
 }
 
@@ -225,6 +263,7 @@ struct vit_model {
   float *patch_b = nullptr, *pos = nullptr, *cls = nullptr, *reg = nullptr, *norm_w = nullptr, *norm_b = nullptr;
   CUtensorMap tm_patch;
   std::vector<BlockW> blocks;
+  std::vector<BlockW> head;  // dino.txt vision head blocks (vit_set_text_head), empty if none
   int* d_status = nullptr;
   int last_launches = 0;
   std::vector<void*> allocs;
@@ -238,11 +277,46 @@ struct vit_model {
 namespace {
 
 struct WsLayout {
-  size_t x, xb, stats, attn, big, total;
+  size_t x, xb, stats, attn, big, pos, total;
 };
 
-WsLayout ws_layout(const vit_model* m, int B) {
-  const size_t M = static_cast<size_t>(B) * m->T, Mp = static_cast<size_t>(B) * m->P;
+// The token geometry of one forward: input H x W, patch grid gh x gw (the convolution's
+// floor), P patch tokens, T = 1 + R + P tokens.  `native` is the size the position embedding
+// was learned for; any other size reads a bicubically resized copy of it from the workspace.
+struct Geom {
+  int H, W, gh, gw, P, T;
+  bool native;
+};
+
+Geom geom_for(const vit_model* m, int H, int W) {
+  Geom g;
+  g.H = H;
+  g.W = W;
+  g.gh = H / m->cfg.patch;
+  g.gw = W / m->cfg.patch;
+  g.P = g.gh * g.gw;
+  g.T = 1 + m->cfg.n_registers + g.P;
+  g.native = (g.gh == m->gh && g.gw == m->gw);
+  return g;
+}
+
+Geom native_geom(const vit_model* m) { return geom_for(m, m->cfg.img_h, m->cfg.img_w); }
+
+vit_status check_geom(const vit_model* m, int B, const Geom& g) {
+  if (g.H < m->cfg.patch || g.W < m->cfg.patch || g.H > 16384 || g.W > 16384) {
+    set_err("image %dx%d outside %d..16384 per side (patch %d)", g.H, g.W, m->cfg.patch, m->cfg.patch);
+    return VIT_E_SHAPE;
+  }
+  // TMA row coordinates and the GEMMs' M are 32-bit
+  if (static_cast<long long>(B) * g.T >= (1LL << 30)) {
+    set_err("batch %d x %d tokens exceeds 2^30 rows", B, g.T);
+    return VIT_E_SHAPE;
+  }
+  return VIT_OK;
+}
+
+WsLayout ws_layout(const vit_model* m, int B, const Geom& g) {
+  const size_t M = static_cast<size_t>(B) * g.T, Mp = static_cast<size_t>(B) * g.P;
   const size_t D = m->cfg.dim, F = m->cfg.mlp_dim;
   WsLayout L;
   size_t off = 0;
@@ -256,6 +330,8 @@ WsLayout ws_layout(const vit_model* m, int B) {
   off = align_up(off + M * D * 2, 1024);
   L.big = off;
   off = align_up(off + std::max(std::max(M * 3 * D, M * F), Mp * static_cast<size_t>(m->Kpad)) * 2, 1024);
+  L.pos = off;
+  if (!g.native) off = align_up(off + (static_cast<size_t>(g.P) + (m->cfg.pos_on_cls ? 1 : 0)) * D * 4, 1024);
   L.total = off;
   return L;
 }
@@ -327,6 +403,44 @@ vit_status validate_cfg(const vit_config* c) {
   return VIT_OK;
 }
 
+// Device copies of one encoder block's weights: the LN-folded QKV and FC1 matrices with their
+// column sums and folded biases, fp32 vectors, and the TMA maps of all four GEMM operands.
+vit_status build_block(vit_model* m, const vit_block_weights& src, BlockW& b, cudaStream_t s) {
+  const int D = m->cfg.dim, F = m->cfg.mlp_dim;
+  vit_status e;
+  if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.qkv_wg), static_cast<size_t>(3) * D * D * 2)) != VIT_OK) return e;
+  if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.qkv_c), static_cast<size_t>(3) * D * 4)) != VIT_OK) return e;
+  if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.qkv_b), static_cast<size_t>(3) * D * 4)) != VIT_OK) return e;
+  if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.fc1_wg), static_cast<size_t>(F) * D * 2)) != VIT_OK) return e;
+  if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.fc1_c), static_cast<size_t>(F) * 4)) != VIT_OK) return e;
+  if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.fc1_b), static_cast<size_t>(F) * 4)) != VIT_OK) return e;
+  fold_ln_weight_kernel<<<3 * D, 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(src.qkv_w), static_cast<const __nv_bfloat16*>(src.qkv_b),
+      static_cast<const __nv_bfloat16*>(src.ln1_w), static_cast<const __nv_bfloat16*>(src.ln1_b), 3 * D, D, b.qkv_wg,
+      b.qkv_c, b.qkv_b);
+  CKL();
+  fold_ln_weight_kernel<<<F, 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(src.fc1_w), static_cast<const __nv_bfloat16*>(src.fc1_b),
+      static_cast<const __nv_bfloat16*>(src.ln2_w), static_cast<const __nv_bfloat16*>(src.ln2_b), F, D, b.fc1_wg,
+      b.fc1_c, b.fc1_b);
+  CKL();
+  b.proj_w = static_cast<const __nv_bfloat16*>(src.proj_w);
+  b.fc2_w = static_cast<const __nv_bfloat16*>(src.fc2_w);
+  if ((e = to_f32(m, src.proj_b, D, &b.proj_b, s)) != VIT_OK) return e;
+  if ((e = to_f32(m, src.ls1, D, &b.ls1, s)) != VIT_OK) return e;
+  if ((e = to_f32(m, src.fc2_b, D, &b.fc2_b, s)) != VIT_OK) return e;
+  if ((e = to_f32(m, src.ls2, D, &b.ls2, s)) != VIT_OK) return e;
+  if (!tmap_2d(&b.tm_qkv[0], b.qkv_wg, D, 3 * D, D, 64, 128) || !tmap_2d(&b.tm_fc1[0], b.fc1_wg, D, F, D, 64, 128) ||
+      !tmap_2d(&b.tm_proj, b.proj_w, D, D, D, 64, m->bn_res) ||
+      !tmap_2d(&b.tm_fc2, b.fc2_w, F, D, F, 64, m->bn_res))
+    return VIT_E_CUDA;
+  b.tm_qkv[1] = b.tm_qkv[0];
+  b.tm_fc1[1] = b.tm_fc1[0];
+  if ((3 * D) % 256 == 0 && !tmap_2d(&b.tm_qkv[1], b.qkv_wg, D, 3 * D, D, 64, 256)) return VIT_E_CUDA;
+  if (F % 256 == 0 && !tmap_2d(&b.tm_fc1[1], b.fc1_wg, D, F, D, 64, 256)) return VIT_E_CUDA;
+  return VIT_OK;
+}
+
 struct Scratch {
   float* x;
   __nv_bfloat16* xb;
@@ -335,11 +449,15 @@ struct Scratch {
   __nv_bfloat16* big;
 };
 
-// The encoder forward on B images read through `src`; outputs per `out`.
-vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs* out, void* ws, size_t ws_bytes,
-                       cudaStream_t s) {
+// The encoder forward on B images read through `src`; outputs per `out`.  With `head` (and a
+// head attached) the dino.txt vision head runs after the backbone and `out->patch_tokens`
+// (fp32) receives its patch rows; the descriptor is not written then.
+vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, const vit_outputs* out, void* ws,
+                       size_t ws_bytes, cudaStream_t s, bool head = false) {
   const vit_config& c = m->cfg;
-  const WsLayout L = ws_layout(m, B);
+  vit_status gst = check_geom(m, B, g);
+  if (gst != VIT_OK) return gst;
+  const WsLayout L = ws_layout(m, B, g);
   if (ws == nullptr || ws_bytes < L.total) {
     set_err("workspace of %zu bytes is smaller than the %zu required for batch %d", ws_bytes, L.total, B);
     return VIT_E_WORKSPACE;
@@ -352,20 +470,34 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs
   Scratch S{reinterpret_cast<float*>(w8 + L.x), reinterpret_cast<__nv_bfloat16*>(w8 + L.xb),
             reinterpret_cast<float2*>(w8 + L.stats), reinterpret_cast<__nv_bfloat16*>(w8 + L.attn),
             reinterpret_cast<__nv_bfloat16*>(w8 + L.big)};
-  const int D = c.dim, F = c.mlp_dim, T = m->T, P = m->P, R = c.n_registers;
+  const int D = c.dim, F = c.mlp_dim, T = g.T, P = g.P, R = c.n_registers;
   const int M = B * T, Mp = B * P;
   int launches = 0;
+  const float* pos = m->pos;
+  if (!g.native) {
+    float* rp = reinterpret_cast<float*>(w8 + L.pos);
+    const long long n = static_cast<long long>(P + (c.pos_on_cls ? 1 : 0)) * D;
+    { const int ps_ = prof_open(m, VIT_K_POS_RESIZE, s);
+    pos_resize_kernel<<<grid_1d(n, 256, m->nsm), 256, 0, s>>>(m->pos, m->gh, m->gw, g.gh, g.gw, D,
+                                                                c.pos_on_cls ? 1 : 0, rp);
+    prof_close(m, ps_, s); }
+    CKL();
+    ++launches;
+    pos = rp;
+  }
 
-  CUtensorMap tm_pe, tm_xb, tm_attn, tm_h, tm_qkv3;
+  CUtensorMap tm_pe, tm_xb, tm_attn, tm_h, tm_qkv3, tm_qkv_out, tm_h_out, tm_x_ep, tm_xb_ep;
   if (!tmap_2d(&tm_pe, S.big, m->Kpad, Mp, m->Kpad, 64, GEMM_BM) || !tmap_2d(&tm_xb, S.xb, D, M, D, 64, GEMM_BM) ||
       !tmap_2d(&tm_attn, S.attn, D, M, D, 64, GEMM_BM) || !tmap_2d(&tm_h, S.big, F, M, F, 64, GEMM_BM) ||
-      !tmap_qkv3d(&tm_qkv3, S.big, B, T, D))
+      !tmap_qkv3d(&tm_qkv3, S.big, B, T, D) || !tmap_out_bf16(&tm_qkv_out, S.big, 3 * D, M, 3 * D) ||
+      !tmap_out_bf16(&tm_h_out, S.big, F, M, F) || !tmap_x_f32(&tm_x_ep, S.x, D, M) ||
+      !tmap_xb_bf16(&tm_xb_ep, S.xb, D, M))
     return VIT_E_CUDA;
 
   // patch embedding: im2col, GEMM with bias + position embedding, token placement
   { const int ps_ = prof_open(m, VIT_K_IM2COL, s);
   im2col_bf16_kernel<<<grid_1d(static_cast<long long>(Mp) * (m->Kpad / 8), 256, m->nsm), 256, 0, s>>>(
-      src, B, c.patch, m->gw, P, m->Kpad, S.big);
+      src, B, c.patch, g.gw, P, m->Kpad, S.big);
   prof_close(m, ps_, s); }
   CKL();
   ++launches;
@@ -377,26 +509,26 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs
     ep.x = S.x;
     ep.xb = S.xb;
     ep.stats_out = S.stats;
-    ep.pos = m->pos;
+    ep.pos = pos;
     ep.P = P;
     ep.T = T;
     ep.R = R;
     ep.pos_off = c.pos_on_cls ? 1 : 0;
     { const int ps_ = prof_open(m, VIT_K_PATCH_GEMM, s);
-    CK(launch_gemm(m->bn_res, EPI_PATCH, tm_pe, m->tm_patch, Mp, D, m->Kpad, ep, m->d_status, s, m->nsm));
+    CK(launch_gemm(m->bn_res, EPI_PATCH, tm_pe, m->tm_patch, tm_pe, tm_pe, Mp, D, m->Kpad, ep, m->d_status, s, m->nsm));
     prof_close(m, ps_, s); }
     ++launches;
   }
   { const int ps_ = prof_open(m, VIT_K_PREFIX, s);
-  prefix_tokens_kernel<<<dim3(m->nt, 1 + R, B), 32, 0, s>>>(m->cls, m->reg, m->pos, c.pos_on_cls, T, D, m->stats_cols,
+  prefix_tokens_kernel<<<dim3(m->nt, 1 + R, B), 32, 0, s>>>(m->cls, m->reg, pos, c.pos_on_cls, T, D, m->stats_cols,
                                                              S.x, S.xb, S.stats);
   prof_close(m, ps_, s); }
   CKL();
   ++launches;
 
-  int tap_i = 0;
-  for (int l = 0; l < c.depth; ++l) {
-    const BlockW& bw = m->blocks[l];
+  // One encoder block ([diagram] "Encoder block"): folded LN1 + QKV, attention, proj + layer
+  // scale + residual, folded LN2 + FC1 + GELU, FC2 + layer scale + residual.
+  auto run_block = [&](const BlockW& bw) -> vit_status {
     // LN1 (folded) + QKV
     {
       const int bn = pick_bn(M, 3 * D, m->nsm);
@@ -410,10 +542,10 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs
       ep.nt_cols = m->stats_cols;
       ep.D = D;
       ep.eps = c.ln_eps;
-      ep.out = S.big;
       ep.ldo = 3 * D;
       { const int ps_ = prof_open(m, VIT_K_QKV_GEMM, s);
-      CK(launch_gemm(bn, EPI_LNFOLD, tm_xb, bw.tm_qkv[bn == 256], M, 3 * D, D, ep, m->d_status, s, m->nsm));
+      CK(launch_gemm(bn, EPI_LNFOLD, tm_xb, bw.tm_qkv[bn == 256], tm_qkv_out, tm_qkv_out, M, 3 * D, D, ep, m->d_status, s,
+                     m->nsm));
       prof_close(m, ps_, s); }
       ++launches;
     }
@@ -432,7 +564,8 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs
       ep.xb = S.xb;
       ep.stats_out = S.stats;
       { const int ps_ = prof_open(m, VIT_K_PROJ_GEMM, s);
-      CK(launch_gemm(m->bn_res, EPI_RESID, tm_attn, bw.tm_proj, M, D, D, ep, m->d_status, s, m->nsm));
+      CK(launch_gemm(m->bn_res, EPI_RESID, tm_attn, bw.tm_proj, tm_x_ep, tm_xb_ep, M, D, D, ep, m->d_status, s,
+                     m->nsm));
       prof_close(m, ps_, s); }
       ++launches;
     }
@@ -449,11 +582,11 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs
       ep.nt_cols = m->stats_cols;
       ep.D = D;
       ep.eps = c.ln_eps;
-      ep.out = S.big;
       ep.ldo = F;
       ep.gelu = 1;
       { const int ps_ = prof_open(m, VIT_K_FC1_GEMM, s);
-      CK(launch_gemm(bn, EPI_LNFOLD, tm_xb, bw.tm_fc1[bn == 256], M, F, D, ep, m->d_status, s, m->nsm));
+      CK(launch_gemm(bn, EPI_LNFOLD, tm_xb, bw.tm_fc1[bn == 256], tm_h_out, tm_h_out, M, F, D, ep, m->d_status, s,
+                     m->nsm));
       prof_close(m, ps_, s); }
       ++launches;
     }
@@ -468,10 +601,18 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs
       ep.xb = S.xb;
       ep.stats_out = S.stats;
       { const int ps_ = prof_open(m, VIT_K_FC2_GEMM, s);
-      CK(launch_gemm(m->bn_res, EPI_RESID, tm_h, bw.tm_fc2, M, D, F, ep, m->d_status, s, m->nsm));
+      CK(launch_gemm(m->bn_res, EPI_RESID, tm_h, bw.tm_fc2, tm_x_ep, tm_xb_ep, M, D, F, ep, m->d_status, s,
+                     m->nsm));
       prof_close(m, ps_, s); }
       ++launches;
     }
+    return VIT_OK;
+  };
+
+  int tap_i = 0;
+  for (int l = 0; l < c.depth; ++l) {
+    const vit_status bst = run_block(m->blocks[l]);
+    if (bst != VIT_OK) return bst;
     if (out && out->hidden)
       CK(cudaMemcpyAsync(out->hidden + static_cast<size_t>(l) * M * D, S.x, static_cast<size_t>(M) * D * 4,
                          cudaMemcpyDeviceToDevice, s));
@@ -487,7 +628,29 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const vit_outputs
       ++tap_i;
     }
   }
-  if (out && (out->desc || out->patch_tokens)) {
+  if (head && !m->head.empty()) {
+    // dino.txt vision head: final norm in place over the whole sequence, the head blocks, then
+    // the head's patch rows (fp32) as the patch tokens
+    const long long rows = static_cast<long long>(M);
+    { const int ps_ = prof_open(m, VIT_K_FINAL_LN, s);
+    final_ln_stream_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(S.x, m->norm_w, m->norm_b, rows, D, c.ln_eps,
+                                                                          m->stats_cols, S.xb, S.stats);
+    prof_close(m, ps_, s); }
+    CKL();
+    ++launches;
+    for (const BlockW& hb : m->head) {
+      const vit_status bst = run_block(hb);
+      if (bst != VIT_OK) return bst;
+    }
+    if (out && out->patch_tokens) {
+      { const int ps_ = prof_open(m, VIT_K_HEAD_OUT, s);
+      patch_rows_kernel<<<grid_1d(static_cast<long long>(B) * P * (D / 4), 256, m->nsm), 256, 0, s>>>(
+          S.x, B, T, R, D, static_cast<float*>(out->patch_tokens));
+      prof_close(m, ps_, s); }
+      CKL();
+      ++launches;
+    }
+  } else if (out && (out->desc || out->patch_tokens)) {
     const long long jobs = static_cast<long long>(B) * (1 + P);
     { const int ps_ = prof_open(m, VIT_K_FINAL_LN, s);
     final_ln_kernel<<<static_cast<int>((jobs + 7) / 8), 256, 0, s>>>(S.x, m->norm_w, m->norm_b, B, T, R, D, c.ln_eps,
@@ -601,38 +764,7 @@ vit_status vit_create(const vit_config* cfg, const vit_weights* w, vit_model** o
     if (!tmap_2d(&m->tm_patch, m->patch_w, m->Kpad, D, m->Kpad, 64, m->bn_res)) return VIT_E_CUDA;
     m->blocks.resize(cfg->depth);
     for (int l = 0; l < cfg->depth; ++l) {
-      const vit_block_weights& src = w->blocks[l];
-      BlockW& b = m->blocks[l];
-      if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.qkv_wg), static_cast<size_t>(3) * D * D * 2)) != VIT_OK) return e;
-      if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.qkv_c), static_cast<size_t>(3) * D * 4)) != VIT_OK) return e;
-      if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.qkv_b), static_cast<size_t>(3) * D * 4)) != VIT_OK) return e;
-      if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.fc1_wg), static_cast<size_t>(F) * D * 2)) != VIT_OK) return e;
-      if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.fc1_c), static_cast<size_t>(F) * 4)) != VIT_OK) return e;
-      if ((e = alloc_dev(m, reinterpret_cast<void**>(&b.fc1_b), static_cast<size_t>(F) * 4)) != VIT_OK) return e;
-      fold_ln_weight_kernel<<<3 * D, 256, 0, s>>>(
-          static_cast<const __nv_bfloat16*>(src.qkv_w), static_cast<const __nv_bfloat16*>(src.qkv_b),
-          static_cast<const __nv_bfloat16*>(src.ln1_w), static_cast<const __nv_bfloat16*>(src.ln1_b), 3 * D, D, b.qkv_wg,
-          b.qkv_c, b.qkv_b);
-      CKL();
-      fold_ln_weight_kernel<<<F, 256, 0, s>>>(
-          static_cast<const __nv_bfloat16*>(src.fc1_w), static_cast<const __nv_bfloat16*>(src.fc1_b),
-          static_cast<const __nv_bfloat16*>(src.ln2_w), static_cast<const __nv_bfloat16*>(src.ln2_b), F, D, b.fc1_wg,
-          b.fc1_c, b.fc1_b);
-      CKL();
-      b.proj_w = static_cast<const __nv_bfloat16*>(src.proj_w);
-      b.fc2_w = static_cast<const __nv_bfloat16*>(src.fc2_w);
-      if ((e = to_f32(m, src.proj_b, D, &b.proj_b, s)) != VIT_OK) return e;
-      if ((e = to_f32(m, src.ls1, D, &b.ls1, s)) != VIT_OK) return e;
-      if ((e = to_f32(m, src.fc2_b, D, &b.fc2_b, s)) != VIT_OK) return e;
-      if ((e = to_f32(m, src.ls2, D, &b.ls2, s)) != VIT_OK) return e;
-      if (!tmap_2d(&b.tm_qkv[0], b.qkv_wg, D, 3 * D, D, 64, 128) || !tmap_2d(&b.tm_fc1[0], b.fc1_wg, D, F, D, 64, 128) ||
-          !tmap_2d(&b.tm_proj, b.proj_w, D, D, D, 64, m->bn_res) ||
-          !tmap_2d(&b.tm_fc2, b.fc2_w, F, D, F, 64, m->bn_res))
-        return VIT_E_CUDA;
-      b.tm_qkv[1] = b.tm_qkv[0];
-      b.tm_fc1[1] = b.tm_fc1[0];
-      if ((3 * D) % 256 == 0 && !tmap_2d(&b.tm_qkv[1], b.qkv_wg, D, 3 * D, D, 64, 256)) return VIT_E_CUDA;
-      if (F % 256 == 0 && !tmap_2d(&b.tm_fc1[1], b.fc1_wg, D, F, D, 64, 256)) return VIT_E_CUDA;
+      if ((e = build_block(m, w->blocks[l], m->blocks[l], s)) != VIT_OK) return e;
     }
     CK(cudaStreamSynchronize(s));
     return VIT_OK;
@@ -660,7 +792,7 @@ vit_status vit_workspace_size(const vit_model* m, int32_t batch, size_t* bytes) 
     set_err("batch %d outside 1..max_batch (%d)", batch, m->cfg.max_batch);
     return VIT_E_SHAPE;
   }
-  *bytes = ws_layout(m, batch).total;
+  *bytes = ws_layout(m, batch, native_geom(m)).total;
   return VIT_OK;
 }
 
@@ -678,7 +810,106 @@ vit_status vit_forward(vit_model* m, const float* images, int32_t B, const vit_o
   if (st != VIT_OK) return st;
   const vit_config& c = m->cfg;
   ImgSrc src{images, 3LL * c.img_h * c.img_w, static_cast<long long>(c.img_h) * c.img_w, c.img_w, 1, 0, 0, 0};
-  return run_forward(m, src, B, out, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+  return run_forward(m, src, B, native_geom(m), out, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+vit_status vit_workspace_size_hw(const vit_model* m, int32_t batch, int32_t H, int32_t W, size_t* bytes) {
+  if (!m || !bytes) {
+    set_err("NULL argument");
+    return VIT_E_INVALID_ARG;
+  }
+  if (batch < 1 || batch > m->cfg.max_batch) {
+    set_err("batch %d outside 1..max_batch (%d)", batch, m->cfg.max_batch);
+    return VIT_E_SHAPE;
+  }
+  const Geom g = geom_for(m, H, W);
+  vit_status st = check_geom(m, batch, g);
+  if (st != VIT_OK) return st;
+  *bytes = ws_layout(m, batch, g).total;
+  return VIT_OK;
+}
+
+vit_status vit_forward_hw(vit_model* m, const float* images, int32_t B, int32_t H, int32_t W, const vit_outputs* out,
+                          void* ws, size_t ws_bytes, vit_stream_t stream) {
+  if (!m || !images || !aligned16(images)) {
+    set_err("model or images NULL / images not 16-byte aligned");
+    return VIT_E_INVALID_ARG;
+  }
+  if (B < 1 || B > m->cfg.max_batch) {
+    set_err("batch %d outside 1..max_batch (%d)", B, m->cfg.max_batch);
+    return VIT_E_SHAPE;
+  }
+  vit_status st = check_outputs(out);
+  if (st != VIT_OK) return st;
+  ImgSrc src{images, 3LL * H * W, static_cast<long long>(H) * W, W, 1, 0, 0, 0};
+  return run_forward(m, src, B, geom_for(m, H, W), out, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+vit_status vit_set_text_head(vit_model* m, const vit_block_weights* blocks, int32_t n_blocks) {
+  if (!m || (n_blocks > 0 && !blocks)) {
+    set_err("NULL argument");
+    return VIT_E_INVALID_ARG;
+  }
+  if (n_blocks < 1 || n_blocks > 8) {
+    set_err("n_blocks %d outside 1..8", n_blocks);
+    return VIT_E_INVALID_ARG;
+  }
+  if (!m->head.empty()) {
+    set_err("a text head is already attached to this model");
+    return VIT_E_INVALID_ARG;
+  }
+  for (int l = 0; l < n_blocks; ++l) {
+    const vit_block_weights& b = blocks[l];
+    const void* ptrs[] = {b.ln1_w, b.ln1_b, b.qkv_w, b.qkv_b, b.proj_w, b.proj_b, b.ls1,
+                          b.ln2_w, b.ln2_b, b.fc1_w, b.fc1_b, b.fc2_w, b.fc2_b, b.ls2};
+    for (const void* p : ptrs)
+      if (!p || !aligned16(p)) {
+        set_err("head block %d: weight pointer NULL or not 16-byte aligned", l);
+        return VIT_E_INVALID_ARG;
+      }
+  }
+  int cur = 0;
+  CK(cudaGetDevice(&cur));
+  if (cur != m->device) {
+    set_err("vit_set_text_head called with device %d current; the model lives on device %d", cur, m->device);
+    return VIT_E_INVALID_ARG;
+  }
+  cudaStream_t s;
+  CK(cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking));
+  std::vector<BlockW> head(n_blocks);
+  vit_status st = VIT_OK;
+  for (int l = 0; l < n_blocks && st == VIT_OK; ++l) st = build_block(m, blocks[l], head[l], s);
+  const cudaError_t se = cudaStreamSynchronize(s);
+  cudaStreamDestroy(s);
+  if (st != VIT_OK) return st;
+  if (se != cudaSuccess) {
+    set_err("vit_set_text_head: %s", cudaGetErrorString(se));
+    return VIT_E_CUDA;
+  }
+  m->head = std::move(head);
+  return VIT_OK;
+}
+
+vit_status vit_forward_text_tokens(vit_model* m, const float* images, int32_t B, int32_t H, int32_t W, float* tokens,
+                                   void* ws, size_t ws_bytes, vit_stream_t stream) {
+  if (!m || !images || !tokens || !aligned16(images) || !aligned16(tokens)) {
+    set_err("model, images or tokens NULL / not 16-byte aligned");
+    return VIT_E_INVALID_ARG;
+  }
+  if (m->head.empty()) {
+    set_err("no text head attached (vit_set_text_head)");
+    return VIT_E_INVALID_ARG;
+  }
+  if (B < 1 || B > m->cfg.max_batch) {
+    set_err("batch %d outside 1..max_batch (%d)", B, m->cfg.max_batch);
+    return VIT_E_SHAPE;
+  }
+  vit_outputs o{};
+  o.patch_tokens = tokens;
+  o.patch_fp32 = 1;
+  ImgSrc src{images, 3LL * H * W, static_cast<long long>(H) * W, W, 1, 0, 0, 0};
+  return run_forward(m, src, B, geom_for(m, H, W), &o, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
+                     /*head=*/true);
 }
 
 vit_status vit_host_workspace_size(const vit_model* m, int32_t batch, size_t* bytes) {
@@ -733,25 +964,61 @@ static int slide_count(int size, int side, int stride) {
   return (size - side + stride - 1) / stride + 1;
 }
 
-vit_status vit_seg_workspace_size(const vit_model* m, int32_t H, int32_t W, int32_t C, int32_t mode, int32_t side,
-                                  int32_t stride, size_t* bytes) {
-  if (!m || !bytes || C < 1) {
-    set_err("NULL argument or C < 1");
+// The view the encoder sees in each zero-shot mode: the whole image, or ny x nx windows of
+// side x side (origins clamped so the last window ends on the border).
+struct SegPlan {
+  Geom g;
+  int ny, nx;
+};
+
+static vit_status seg_plan(const vit_model* m, int32_t H, int32_t W, int32_t C, int32_t mode, int32_t side, int32_t stride,
+                    SegPlan* p) {
+  if (C < 1) {
+    set_err("C (%d) must be >= 1", C);
     return VIT_E_INVALID_ARG;
   }
-  int nwin = 1;
   if (mode == VIT_SEG_SLIDE) {
-    if (stride < 1 || side < 1) {
-      set_err("side and stride must be positive");
+    if (stride < 1 || side < m->cfg.patch) {
+      set_err("slide: stride must be >= 1 and side >= the patch size %d", m->cfg.patch);
       return VIT_E_INVALID_ARG;
     }
-    nwin = slide_count(H, side, stride) * slide_count(W, side, stride);
+    if (H < side || W < side) {
+      set_err("slide: window side %d must fit in the image %dx%d", side, H, W);
+      return VIT_E_SHAPE;
+    }
+    p->ny = slide_count(H, side, stride);
+    p->nx = slide_count(W, side, stride);
+    p->g = geom_for(m, side, side);
+  } else if (mode == VIT_SEG_WHOLE) {
+    p->ny = p->nx = 1;
+    p->g = geom_for(m, H, W);
+  } else {
+    set_err("mode must be VIT_SEG_WHOLE or VIT_SEG_SLIDE");
+    return VIT_E_INVALID_ARG;
   }
-  size_t fw = 0;
-  vit_status st = vit_workspace_size(m, nwin, &fw);
+  const int nwin = p->ny * p->nx;
+  if (nwin > m->cfg.max_batch) {
+    set_err("%d windows exceed max_batch (%d)", nwin, m->cfg.max_batch);
+    return VIT_E_SHAPE;
+  }
+  return check_geom(m, nwin, p->g);
+}
+
+static size_t seg_head_bytes(const vit_model* m, const SegPlan& p, int C) {
+  const size_t rows = static_cast<size_t>(p.ny) * p.nx * p.g.P;
+  return align_up(rows * m->cfg.dim * 4, 1024) + align_up(rows * 4, 1024) + align_up(rows * C * 4, 1024);
+}
+
+vit_status vit_seg_workspace_size(const vit_model* m, int32_t H, int32_t W, int32_t C, int32_t mode, int32_t side,
+                                  int32_t stride, size_t* bytes) {
+  if (!m || !bytes) {
+    set_err("NULL argument");
+    return VIT_E_INVALID_ARG;
+  }
+  SegPlan p;
+  vit_status st = seg_plan(m, H, W, C, mode, side, stride, &p);
   if (st != VIT_OK) return st;
-  const size_t rows = static_cast<size_t>(nwin) * m->P;
-  *bytes = align_up(rows * m->cfg.dim * 4, 1024) + align_up(rows * 4, 1024) + align_up(rows * C * 4, 1024) + fw;
+  *bytes = seg_head_bytes(m, p, C) + ws_layout(m, p.ny * p.nx, p.g).total;
   return VIT_OK;
 }
 
@@ -763,35 +1030,17 @@ vit_status vit_seg_zero_shot(vit_model* m, const float* image, int32_t H, int32_
     return VIT_E_INVALID_ARG;
   }
   const vit_config& c = m->cfg;
-  int ny = 1, nx = 1, g = 0;
-  if (mode == VIT_SEG_SLIDE) {
-    if (side != c.img_h || side != c.img_w || H < side || W < side) {
-      set_err("slide: side (%d) must equal the model input %dx%d and fit in the image %dx%d", side, c.img_h, c.img_w, H,
-              W);
-      return VIT_E_SHAPE;
-    }
-    ny = slide_count(H, side, stride);
-    nx = slide_count(W, side, stride);
-    g = m->gh;
-  } else if (mode == VIT_SEG_WHOLE) {
-    if (H != c.img_h || W != c.img_w) {
-      set_err("whole: image %dx%d must equal the model input %dx%d (no position-embedding resize)", H, W, c.img_h,
-              c.img_w);
-      return VIT_E_UNSUPPORTED;
-    }
-  } else {
-    set_err("mode must be VIT_SEG_WHOLE or VIT_SEG_SLIDE");
-    return VIT_E_INVALID_ARG;
-  }
-  size_t need = 0;
-  vit_status st = vit_seg_workspace_size(m, H, W, C, mode, side, stride, &need);
+  SegPlan plan;
+  vit_status st = seg_plan(m, H, W, C, mode, side, stride, &plan);
   if (st != VIT_OK) return st;
+  const size_t head = seg_head_bytes(m, plan, C);
+  const size_t need = head + ws_layout(m, plan.ny * plan.nx, plan.g).total;
   if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) {
     set_err("seg workspace must be >= %zu bytes and 256-byte aligned", need);
     return VIT_E_WORKSPACE;
   }
-  const int nwin = ny * nx;
-  const size_t rows = static_cast<size_t>(nwin) * m->P;
+  const int ny = plan.ny, nx = plan.nx, nwin = ny * nx, P = plan.g.P;
+  const size_t rows = static_cast<size_t>(nwin) * P;
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   float* tok = reinterpret_cast<float*>(w8);
   size_t off = align_up(rows * c.dim * 4, 1024);
@@ -806,7 +1055,7 @@ vit_status vit_seg_zero_shot(vit_model* m, const float* image, int32_t H, int32_
   vit_outputs o{};
   o.patch_tokens = tok;
   o.patch_fp32 = 1;
-  st = run_forward(m, src, nwin, &o, w8 + off, ws_bytes - off, s);
+  st = run_forward(m, src, nwin, plan.g, &o, w8 + off, ws_bytes - off, s, /*head=*/true);
   if (st != VIT_OK) return st;
   int launches = m->last_launches;
   { const int ps_ = prof_open(m, VIT_K_SEG_NORM, s);
@@ -815,19 +1064,20 @@ vit_status vit_seg_zero_shot(vit_model* m, const float* image, int32_t H, int32_
   CKL();
   dim3 cg(static_cast<unsigned>((rows + 63) / 64), static_cast<unsigned>((C + 63) / 64));
   { const int ps_ = prof_open(m, VIT_K_SEG_COS, s);
-  cos_gemm_kernel<<<cg, 256, 0, s>>>(tok, inv, text, m->P, static_cast<long long>(rows), C, c.dim, cosm);
+  cos_gemm_kernel<<<cg, 256, 0, s>>>(tok, inv, text, P, static_cast<long long>(rows), C, c.dim, cosm);
   prof_close(m, ps_, s); }
   CKL();
   launches += 2;
   const long long pix = static_cast<long long>(H) * W;
   if (mode == VIT_SEG_SLIDE) {
     { const int ps_ = prof_open(m, VIT_K_SEG_MAP, s);
-    seg_slide_kernel<<<static_cast<int>((pix + 127) / 128), 128, 0, s>>>(cosm, C, g, H, W, side, stride, ny, nx, probs,
-                                                                         labels);
+    seg_slide_kernel<<<static_cast<int>((pix + 127) / 128), 128, 0, s>>>(cosm, C, plan.g.gh, H, W, side, stride, ny,
+                                                                         nx, probs, labels);
     prof_close(m, ps_, s); }
   } else {
     { const int ps_ = prof_open(m, VIT_K_SEG_MAP, s);
-    seg_whole_kernel<<<static_cast<int>((pix + 127) / 128), 128, 0, s>>>(cosm, C, m->gh, m->gw, H, W, probs, labels);
+    seg_whole_kernel<<<static_cast<int>((pix + 127) / 128), 128, 0, s>>>(cosm, C, plan.g.gh, plan.g.gw, H, W, probs,
+                                                                         labels);
     prof_close(m, ps_, s); }
   }
   CKL();
@@ -909,16 +1159,16 @@ vit_status vit_stage_linear(const void* A, const void* W, const float* bias, int
   CK(cudaGetDevice(&dev));
   const int nsm = device_sms(dev);
   const int bn = pick_bn(M, N, nsm);
-  CUtensorMap ta, tb;
-  if (!tmap_2d(&ta, A, K, M, K, 64, GEMM_BM) || !tmap_2d(&tb, W, K, N, K, 64, bn)) return VIT_E_CUDA;
+  CUtensorMap ta, tb, to;
+  if (!tmap_2d(&ta, A, K, M, K, 64, GEMM_BM) || !tmap_2d(&tb, W, K, N, K, 64, bn) || !tmap_out_bf16(&to, out, N, M, N))
+    return VIT_E_CUDA;
   EpiParams ep{};
   ep.M = M;
   ep.N = N;
   ep.bias = bias;
   ep.gelu = gelu;
-  ep.out = static_cast<__nv_bfloat16*>(out);
   ep.ldo = N;
-  CK(launch_gemm(bn, EPI_BIAS, ta, tb, M, N, K, ep, status, reinterpret_cast<cudaStream_t>(stream), nsm));
+  CK(launch_gemm(bn, EPI_BIAS, ta, tb, to, to, M, N, K, ep, status, reinterpret_cast<cudaStream_t>(stream), nsm));
   return VIT_OK;
 }
 
@@ -936,6 +1186,26 @@ vit_status vit_stage_attention(const void* qkv, int32_t B, int32_t T, int32_t he
   if (!tmap_qkv3d(&tm, qkv, B, T, heads * 64)) return VIT_E_CUDA;
   CK(launch_attention(tm, static_cast<const __nv_bfloat16*>(qkv), B, T, heads, static_cast<__nv_bfloat16*>(out), status,
                       reinterpret_cast<cudaStream_t>(stream)));
+  return VIT_OK;
+}
+
+vit_status vit_stage_pos_resize(const float* pos, int32_t gh0, int32_t gw0, int32_t gh, int32_t gw, int32_t D,
+                                int32_t pos_on_cls, float* out, vit_stream_t stream) {
+  if (!pos || !out) {
+    set_err("NULL pointer");
+    return VIT_E_INVALID_ARG;
+  }
+  if (gh0 < 1 || gw0 < 1 || gh < 1 || gw < 1 || D < 1 || gh > 4096 || gw > 4096 || gh0 > 4096 || gw0 > 4096) {
+    set_err("grids must be 1..4096 per side and D >= 1");
+    return VIT_E_SHAPE;
+  }
+  int dev = 0, nsm = 1;
+  CK(cudaGetDevice(&dev));
+  CK(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+  const long long n = static_cast<long long>(gh * gw + (pos_on_cls ? 1 : 0)) * D;
+  pos_resize_kernel<<<grid_1d(n, 256, nsm), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      pos, gh0, gw0, gh, gw, D, pos_on_cls ? 1 : 0, out);
+  CKL();
   return VIT_OK;
 }
 
@@ -987,7 +1257,7 @@ extern "C" vit_status vit_forward_noalloc(vit_model* m, const float* images, int
   }
   vit_status st = check_outputs(out);
   if (st != VIT_OK) return st;
-  const size_t need = ws_layout(m, B).total;
+  const size_t need = ws_layout(m, B, native_geom(m)).total;
   if (need > kNoAllocScratchBytes) {
     set_err("vit_forward_noalloc: batch %d of this model needs %zu bytes of scratch, more than the fixed %zu "
             "bytes; use vit_forward with a caller-provided workspace",
@@ -999,5 +1269,5 @@ extern "C" vit_status vit_forward_noalloc(vit_model* m, const float* images, int
   if (st != VIT_OK) return st;
   const vit_config& c = m->cfg;
   ImgSrc src{images, 3LL * c.img_h * c.img_w, static_cast<long long>(c.img_h) * c.img_w, c.img_w, 1, 0, 0, 0};
-  return run_forward(m, src, B, out, ws, kNoAllocScratchBytes, reinterpret_cast<cudaStream_t>(stream));
+  return run_forward(m, src, B, native_geom(m), out, ws, kNoAllocScratchBytes, reinterpret_cast<cudaStream_t>(stream));
 }
