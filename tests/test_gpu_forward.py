@@ -138,3 +138,17 @@ def test_other_widths(name):
     g = run_gpu(spec, w, im)
     ref = O.forward(im, w, spec, record_hidden=True)
     assert_forward_parity(g, ref, spec, [0, 1])
+
+
+def test_vitb14_224_b64_paired_gemms():
+    """Batch 64 of ViT-B/14 (M = 16,448 rows): every block GEMM runs on paired 256 x 256 tiles."""
+    need_cuda()
+    spec = S.PRESETS["vitb14_224"]
+    w = S.make_weights(spec, 73)
+    im = S.make_images(spec, 64, 74)
+    keep = [0, 37, 63]
+    g = run_gpu(spec, w, im, keep=keep)
+    assert g["hidden_finite"]
+    ref = O.forward(im, w, spec, record_hidden=True, image_indices=keep)
+    assert_forward_parity(g, ref, spec, keep)
+

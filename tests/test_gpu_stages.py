@@ -24,7 +24,10 @@ def _ref_linear(A, W, b, gelu):
     (446, 1152, 384, False),    # ViT-S/16 QKV shape
     (446, 1536, 384, True),     # ViT-S/16 FC1 with GELU
     (1000, 1024, 4096, False),  # long K (FC2-like), ragged M
-    (5000, 4096, 1024, True),   # 256-column tiles (enough tiles to fill the SMs)
+    (5000, 4096, 1024, True),   # paired 256 x 256 tiles (2-CTA clusters), GELU
+    (20000, 1024, 1024, False), # paired tiles; last tile: 32 rows on the first CTA, none on the second
+    (10184, 3072, 1024, False), # paired tiles; last tile: 256 + 72 rows
+    (4096, 768, 3072, False),   # paired tiles, N = 3 x 256, long K
 ])
 def test_linear_matches_oracle(M, N, K, gelu):
     need_cuda()

@@ -18,6 +18,7 @@
 // The double-buffered accumulator lets the epilogue of tile i overlap the MMAs of tile i+1.
 #pragma once
 
+#include "cluster.cuh"
 #include "common.cuh"
 
 namespace vit {
@@ -501,6 +502,261 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Paired variant: a 2-CTA cluster computes one 256 x 256 tile with M = 256 tcgen05.mma
+// (cta_group::2).  Each CTA loads its 128 rows of A and its 128 of the 256 B rows (16 KB + 16 KB
+// per 64-deep stage instead of 16 KB + 32 KB), so per SM the tensor core consumes 131 instead of
+// 87 FLOP per byte brought into shared memory.  Roles as in gemm_bf16_tc_kernel, with:
+//   * both CTAs' producers fill their own stages and count the bytes on the leader's (rank 0)
+//     full barrier; only the leader arms it (with both CTAs' bytes);
+//   * the leader's lane issues the MMAs and commits stage / accumulator / final completion to
+//     the barriers at the same offsets in both CTAs (multicast commit);
+//   * each CTA's epilogue reads its own 128 accumulator rows from its own TMEM and releases the
+//     accumulator by arriving (one arrive per warp) on the leader's tempty barrier.
+// No TMA load uses cluster multicast.
+template <int MODE>
+struct PairCfg {
+  static constexpr int BN = 256;
+  static constexpr int STAGES = (MODE == EPI_RESID) ? 4 : 6;
+  static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
+  static constexpr int B_BYTES = (BN / 2) * GEMM_BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_WARP_BYTES = GemmCfg<256, MODE>::EPI_WARP_BYTES;
+  static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
+  static constexpr int OFF_BAR = OFF_EPI + GEMM_EPI_WARPS * EPI_WARP_BYTES;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(MODE != EPI_PATCH, "the patch GEMM runs unpaired");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(8 * (2 * STAGES + 5 + 2 * GEMM_EPI_WARPS) + 8 <= BAR_BYTES, "barrier area");
+};
+
+__device__ __forceinline__ int ld_shared_cluster_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// Bounded pause (nanoseconds on the global timer) for copies whose completion this CTA cannot
+// observe itself (its loads are counted on the peer's barrier); used only after an abort.
+__device__ __forceinline__ void grace_wait_ns(unsigned long long ns) {
+  const unsigned long long t0 = global_ns();
+  while (global_ns() - t0 < ns) {
+  }
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmO1, const __grid_constant__ CUtensorMap tmO2, int M, int N,
+                     int K, EpiParams ep, int* gstatus) {
+  using Cfg = PairCfg<MODE>;
+  constexpr int BN = Cfg::BN;
+  constexpr int STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+  uint8_t* sEpi = smem + Cfg::OFF_EPI;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint64_t* xfull = mma_done + 1;  // [GEMM_EPI_WARPS][2] (RESID)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(xfull + 2 * GEMM_EPI_WARPS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+
+  if (threadIdx.x == 0) {
+    *abort_flag = (*reinterpret_cast<volatile int*>(gstatus) != 0) ? 1 : 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * GEMM_EPI_WARPS);  // one arrive per epilogue warp of each CTA
+    }
+    mbar_init(mma_done, 1);
+    for (int i = 0; i < 2 * GEMM_EPI_WARPS; ++i) mbar_init(&xfull[i], 1);
+    fence_mbar_init_cluster();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmO1);
+    if (MODE == EPI_RESID) tma_prefetch_desc(&tmO2);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, Cfg::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  // the leader's view decides for both CTAs
+  const bool skip = ld_shared_cluster_s32(mapa_shared(smem_u32(const_cast<int*>(abort_flag)), 0)) != 0;
+
+  const int num_m = (M + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
+  const int num_n = N / BN;
+  const int num_tiles = num_m * num_n;
+  const int KB = K / GEMM_BK;
+  const int cid = static_cast<int>(blockIdx.x >> 1);
+  const int ncl = static_cast<int>(gridDim.x >> 1);
+
+  if (!skip && warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer (both CTAs)
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued_parity[STAGES];
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
+    bool issued_any = false;
+    for (int tile = cid; tile < num_tiles; tile += ncl) {
+      const int mb = tile / num_n;
+      const int nb = tile - mb * num_n;
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 5)) {
+          ok = false;
+          break;
+        }
+        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::STAGE_BYTES);
+        const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+        tma_load_2d_pair(sA + stage * Cfg::A_BYTES, &tmA, kb * GEMM_BK, mb * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM,
+                         bar);
+        tma_load_2d_pair(sB + stage * Cfg::B_BYTES, &tmB, kb * GEMM_BK, nb * BN + static_cast<int>(rank) * (BN / 2), bar);
+        issued_parity[stage] = static_cast<int>(phase);
+        issued_any = true;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+    }
+    if (*abort_flag) {
+      // let every issued copy land before the CTA can exit: the leader sees both CTAs' bytes on
+      // its full barriers; the peer cannot observe its own completions and pauses instead
+      if (leader) {
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_parity[s] >= 0) mbar_wait_drain(&full[s], static_cast<uint32_t>(issued_parity[s]));
+      } else if (issued_any) {
+        grace_wait_ns(200000ull);
+      }
+    }
+  } else if (!skip && warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer (leader)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(2 * GEMM_BM, BN, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = cid; tile < num_tiles && ok; tile += ncl) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 6)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 7)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * Cfg::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < GEMM_BK / 16; ++k) {
+            tc_mma_ss_pair(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024), sdesc_sw128(b0 + k * 32, 16, 1024), idesc,
+                           (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair_mc(&empty[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(&tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      tc_commit_pair_mc(mma_done, 0x3);
+    }
+    __syncwarp();
+  } else if (!skip && warp >= 2) {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int e = warp - 2;
+    const int q = warp & 3;
+    const int half = e >> 2;
+    uint8_t* wbuf = sEpi + e * Cfg::EPI_WARP_BYTES;
+    uint64_t* wxfull = xfull + 2 * e;
+    uint32_t xph[2] = {0u, 0u};
+    bool xpending[2] = {false, false};
+    bool ok = true;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cid; tile < num_tiles && ok; tile += ncl) {
+      const int mb = tile / num_n;
+      const int nb = tile - mb * num_n;
+      const int row0 = mb * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM + q * 32;
+      const int n0 = nb * BN + half * (BN / 2);
+      if (MODE == EPI_RESID && lane == 0) {
+        tma_store_wait_read0();
+        mbar_arrive_expect_tx(&wxfull[0], 4096);
+        tma_load_2d(wbuf, &tmO1, n0, row0, &wxfull[0]);
+        xpending[0] = true;
+      }
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 8)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN + half * (BN / 2));
+      __syncwarp();
+      if (MODE == EPI_RESID) {
+        epilogue_resid<BN>(ep, &tmO1, &tmO2, taddr, row0, n0, wbuf, wbuf + 8192, wxfull, xph, xpending, abort_flag,
+                           gstatus, ok);
+        if (!ok) break;
+      } else {
+        epilogue_store_bf16<BN, MODE>(ep, &tmO1, taddr, row0, n0, wbuf);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    if (lane == 0) {
+      if (MODE == EPI_RESID) {
+        for (int bb = 0; bb < 2; ++bb)
+          if (xpending[bb]) mbar_wait_drain(&wxfull[bb], xph[bb]);
+      }
+      tma_store_wait0();
+    }
+    __syncwarp();
+  }
+
+  // ---------------------------------------------------------------- teardown
+  __syncthreads();
+  if (warp == 1 && !skip && lane == 0) {
+    // every MMA of the pair (which reads this CTA's shared memory and writes its TMEM) is done
+    mbar_wait_drain(mma_done, 0);
+  }
+  __syncwarp();
+  tc_fence_before();
+  // no CTA leaves while the other may still signal its barriers or use its TMEM
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
   }
 }
 

@@ -191,11 +191,62 @@ cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b, const CUte
   return cudaGetLastError();
 }
 
+// Tile code for the paired kernel (a 2-CTA cluster per 256 x 256 tile); its B map has 128-row boxes.
+constexpr int BN_PAIR = 512;
+
+template <int MODE>
+cudaError_t launch_gemm_pair_t(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o1,
+                               const CUtensorMap& o2, int M, int N, int K, const EpiParams& ep, int* st, cudaStream_t s,
+                               int nsm) {
+  static std::atomic<uint64_t> attr_done{0};
+  static std::atomic<int> max_clusters{0};
+  constexpr int smem = PairCfg<MODE>::SMEM_BYTES;
+  cudaError_t e = set_smem_attr_once(gemm_pair_kernel<MODE>, smem, attr_done);
+  if (e != cudaSuccess) return e;
+  int mc = max_clusters.load();
+  if (mc == 0) {
+    // how many 2-CTA clusters of this size fit on the device at once (the GPC layout can leave
+    // an SM without a partner); the persistent grid never exceeds it
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (nsm / 2), 1, 1);
+    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<MODE>, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = nsm / 2;
+    }
+    mc = std::max(1, std::min(n, nsm / 2));
+    max_clusters.store(mc);
+  }
+  const int tiles = ((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * (N / 256);
+  const int clusters = std::max(1, std::min(tiles, mc));
+  gemm_pair_kernel<MODE><<<2 * clusters, GEMM_THREADS, smem, s>>>(a, b, o1, o2, M, N, K, ep, st);
+  return cudaGetLastError();
+}
+
 // o1 / o2: BIAS, LNFOLD: o1 = bf16 output map (tmap_out_bf16); RESID: o1 = x (tmap_x_f32),
-// o2 = xb (tmap_xb_bf16); PATCH: not read (any valid map).
+// o2 = xb (tmap_xb_bf16); PATCH: not read (any valid map).  bn: 128 or 256 (one CTA per tile,
+// B map boxes of bn rows) or BN_PAIR (B map boxes of 128 rows; not for PATCH).
 cudaError_t launch_gemm(int bn, int mode, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o1,
                         const CUtensorMap& o2, int M, int N, int K, const EpiParams& ep, int* st, cudaStream_t s,
                         int nsm) {
+  if (bn == BN_PAIR) {
+    switch (mode) {
+      case EPI_BIAS: return launch_gemm_pair_t<EPI_BIAS>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
+      case EPI_LNFOLD: return launch_gemm_pair_t<EPI_LNFOLD>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
+      case EPI_RESID: return launch_gemm_pair_t<EPI_RESID>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   if (bn == 256) {
     switch (mode) {
       case EPI_BIAS: return launch_gemm_t<256, EPI_BIAS>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
@@ -228,11 +279,22 @@ int grid_1d(long long work, int block, int nsm) {
   return static_cast<int>(std::max(1LL, std::min(g, static_cast<long long>(nsm) * 32)));
 }
 
-// GEMM N-tile: 256 columns when N allows it and the tile count still fills the SMs.
+// GEMM tiling: the paired 256 x 256 tile when N allows it and the pairs still fill the SMs,
+// else 128 x 256 per CTA when that fills them, else 128 x 128.
 int pick_bn(int M, int N, int nsm) {
   if (N % 256 != 0) return 128;
+  const long long pairs = static_cast<long long>((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * (N / 256);
+  if (pairs >= nsm / 2) return BN_PAIR;
   const long long tiles256 = static_cast<long long>((M + GEMM_BM - 1) / GEMM_BM) * (N / 256);
   return tiles256 >= nsm ? 256 : 128;
+}
+
+// Residual GEMMs (proj, FC2): N = D; the paired tile when it fills the SMs, else bn_res (whose
+// half-width fixes the statistics groups, 128 columns for both 256-wide choices).
+int pick_bn_res(int M, int D, int bn_res, int nsm) {
+  if (bn_res != 256) return bn_res;
+  const long long pairs = static_cast<long long>((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * (D / 256);
+  return pairs >= nsm / 2 ? BN_PAIR : 256;
 }
 
 }  // namespace
@@ -253,6 +315,7 @@ struct BlockW {
   float* ls2;
   CUtensorMap tm_qkv[2], tm_fc1[2];  // [0]: box rows 128, [1]: 256
   CUtensorMap tm_proj, tm_fc2;       // box rows bn_res
+  CUtensorMap tm_proj_h, tm_fc2_h;   // box rows 128 (paired tiles)
 };
 
 struct vit_model {
@@ -432,7 +495,8 @@ vit_status build_block(vit_model* m, const vit_block_weights& src, BlockW& b, cu
   if ((e = to_f32(m, src.ls2, D, &b.ls2, s)) != VIT_OK) return e;
   if (!tmap_2d(&b.tm_qkv[0], b.qkv_wg, D, 3 * D, D, 64, 128) || !tmap_2d(&b.tm_fc1[0], b.fc1_wg, D, F, D, 64, 128) ||
       !tmap_2d(&b.tm_proj, b.proj_w, D, D, D, 64, m->bn_res) ||
-      !tmap_2d(&b.tm_fc2, b.fc2_w, F, D, F, 64, m->bn_res))
+      !tmap_2d(&b.tm_fc2, b.fc2_w, F, D, F, 64, m->bn_res) || !tmap_2d(&b.tm_proj_h, b.proj_w, D, D, D, 64, 128) ||
+      !tmap_2d(&b.tm_fc2_h, b.fc2_w, F, D, F, 64, 128))
     return VIT_E_CUDA;
   b.tm_qkv[1] = b.tm_qkv[0];
   b.tm_fc1[1] = b.tm_fc1[0];
@@ -563,9 +627,10 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
       ep.x = S.x;
       ep.xb = S.xb;
       ep.stats_out = S.stats;
+      const int bnr = pick_bn_res(M, D, m->bn_res, m->nsm);
       { const int ps_ = prof_open(m, VIT_K_PROJ_GEMM, s);
-      CK(launch_gemm(m->bn_res, EPI_RESID, tm_attn, bw.tm_proj, tm_x_ep, tm_xb_ep, M, D, D, ep, m->d_status, s,
-                     m->nsm));
+      CK(launch_gemm(bnr, EPI_RESID, tm_attn, bnr == BN_PAIR ? bw.tm_proj_h : bw.tm_proj, tm_x_ep, tm_xb_ep, M, D, D, ep,
+                     m->d_status, s, m->nsm));
       prof_close(m, ps_, s); }
       ++launches;
     }
@@ -600,9 +665,10 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
       ep.x = S.x;
       ep.xb = S.xb;
       ep.stats_out = S.stats;
+      const int bnr = pick_bn_res(M, D, m->bn_res, m->nsm);
       { const int ps_ = prof_open(m, VIT_K_FC2_GEMM, s);
-      CK(launch_gemm(m->bn_res, EPI_RESID, tm_h, bw.tm_fc2, tm_x_ep, tm_xb_ep, M, D, F, ep, m->d_status, s,
-                     m->nsm));
+      CK(launch_gemm(bnr, EPI_RESID, tm_h, bnr == BN_PAIR ? bw.tm_fc2_h : bw.tm_fc2, tm_x_ep, tm_xb_ep, M, D, F, ep,
+                     m->d_status, s, m->nsm));
       prof_close(m, ps_, s); }
       ++launches;
     }
@@ -1160,7 +1226,8 @@ vit_status vit_stage_linear(const void* A, const void* W, const float* bias, int
   const int nsm = device_sms(dev);
   const int bn = pick_bn(M, N, nsm);
   CUtensorMap ta, tb, to;
-  if (!tmap_2d(&ta, A, K, M, K, 64, GEMM_BM) || !tmap_2d(&tb, W, K, N, K, 64, bn) || !tmap_out_bf16(&to, out, N, M, N))
+  if (!tmap_2d(&ta, A, K, M, K, 64, GEMM_BM) || !tmap_2d(&tb, W, K, N, K, 64, bn == BN_PAIR ? 128 : bn) ||
+      !tmap_out_bf16(&to, out, N, M, N))
     return VIT_E_CUDA;
   EpiParams ep{};
   ep.M = M;
