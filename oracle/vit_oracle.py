@@ -55,7 +55,8 @@ __all__ = [
     "bicubic_resize", "resize_pos_embed", "bf16_round", "to_f64_weights", "patch_embed", "assemble_tokens", "layer_norm", "gelu",
     "attention", "attention_probs", "encoder_block", "forward", "l2_normalize", "cos_map",
     "bilinear_resize", "window_origins", "overlap_counts", "seg_slide_from_tokens",
-    "seg_whole_from_tokens", "seg_slide", "seg_whole", "text_head", "HEAD_DIM",
+    "seg_whole_from_tokens", "seg_slide", "seg_whole", "text_head", "conv2d", "channel_layer_norm", "silu",
+    "group_norm", "dense_projector", "dense_task_head", "dense_head", "HEAD_DIM",
 ]
 
 HEAD_DIM = 64
@@ -460,3 +461,106 @@ def seg_whole(image, weights, spec, text, head_blocks=None):
     tok = o["patch_tokens"][0] if head_blocks is None else text_head(o["final_tokens"], head_blocks, spec)[0]
     scores, labels = seg_whole_from_tokens(tok, txt, img.shape[2], img.shape[3], o["grid"])
     return scores, labels, tok
+
+
+# ---------------------------------------------------------------------------------------------
+# Dense head on the taps ([diagram] "Projector P4", "Projector Bottleneck", "Projector output
+# ConvX", "Task head"; the LibreYOLO DINOv2 configuration): the four tap maps [D, g, g] are
+# concatenated, projected by a C2f block (1x1 conv, channel LayerNorm, SiLU; split into two
+# halves; three chained bottlenecks of two 3x3 conv / channel LN / SiLU each, no residual; all
+# five pieces concatenated; 1x1 conv / channel LN / SiLU; a final channel LN), then the semantic
+# head: lateral 1x1 conv, 3x3 smoothing conv, GroupNorm(32), GELU, dropout (identity at
+# inference), 1x1 prediction conv to the class logits, bilinear resize to the input size.
+# Readings: channel LayerNorm normalises each pixel over its channels with the biased variance
+# and eps = 1e-6 (the only LayerNorm eps the diagram prints); GroupNorm uses eps = 1e-5 (the
+# library default; none is printed); the prediction conv carries a bias (the diagram marks
+# bias=False only on the projector's convs).
+# ---------------------------------------------------------------------------------------------
+CHANNEL_LN_EPS = 1e-6
+GROUP_NORM_EPS = 1e-5
+
+
+def conv2d(x: np.ndarray, w: np.ndarray, b: Optional[np.ndarray], pad: int) -> np.ndarray:
+    """x [C, H, W], w [O, C, k, k], stride 1, zero padding `pad` -> [O, H', W'].  Written as
+    the sum over kernel taps (ky, kx) of W[:, :, ky, kx] times the shifted input."""
+    C, H, W = x.shape
+    O, _, k, _ = w.shape
+    xp = np.pad(x, ((0, 0), (pad, pad), (pad, pad)))
+    Ho, Wo = H + 2 * pad - k + 1, W + 2 * pad - k + 1
+    out = np.zeros((O, Ho * Wo))
+    for ky in range(k):
+        for kx in range(k):
+            out += w[:, :, ky, kx] @ xp[:, ky:ky + Ho, kx:kx + Wo].reshape(C, Ho * Wo)
+    if b is not None:
+        out += b[:, None]
+    return out.reshape(O, Ho, Wo)
+
+
+def channel_layer_norm(x: np.ndarray, g: np.ndarray, b: np.ndarray, eps: float = CHANNEL_LN_EPS) -> np.ndarray:
+    """x [C, H, W]: each pixel's C values normalised (biased variance), then g * . + b."""
+    mu = x.mean(axis=0, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=0, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * g[:, None, None] + b[:, None, None]
+
+
+def silu(x: np.ndarray) -> np.ndarray:
+    return x / (1.0 + np.exp(-x))
+
+
+def group_norm(x: np.ndarray, groups: int, g: np.ndarray, b: np.ndarray, eps: float = GROUP_NORM_EPS) -> np.ndarray:
+    """x [C, H, W]: each group of C/groups channels normalised over its channels and pixels."""
+    C, H, W = x.shape
+    xg = x.reshape(groups, -1)
+    mu = xg.mean(axis=1, keepdims=True)
+    var = ((xg - mu) ** 2).mean(axis=1, keepdims=True)
+    y = ((xg - mu) / np.sqrt(var + eps)).reshape(C, H, W)
+    return y * g[:, None, None] + b[:, None, None]
+
+
+def _conv_ln_silu(x, w, ln_g, ln_b, pad):
+    return silu(channel_layer_norm(conv2d(x, w, None, pad), ln_g, ln_b))
+
+
+def dense_projector(taps: Sequence[np.ndarray], hw: Dict[str, np.ndarray]) -> np.ndarray:
+    """Projector P4 on one image: taps = four [D, g, g] maps -> [256, g, g]."""
+    x = np.concatenate(list(taps), axis=0)
+    y = _conv_ln_silu(x, hw["cv1_w"], hw["cv1_ln_w"], hw["cv1_ln_b"], 0)
+    half = y.shape[0] // 2
+    pieces = [y[:half], y[half:]]
+    cur = pieces[1]
+    for i in range(3):
+        t = _conv_ln_silu(cur, hw["bn_w"][2 * i], hw["bn_ln_w"][2 * i], hw["bn_ln_b"][2 * i], 1)
+        cur = _conv_ln_silu(t, hw["bn_w"][2 * i + 1], hw["bn_ln_w"][2 * i + 1], hw["bn_ln_b"][2 * i + 1], 1)
+        pieces.append(cur)
+    z = _conv_ln_silu(np.concatenate(pieces, axis=0), hw["cv2_w"], hw["cv2_ln_w"], hw["cv2_ln_b"], 0)
+    return channel_layer_norm(z, hw["out_ln_w"], hw["out_ln_b"])
+
+
+def dense_task_head(p4: np.ndarray, hw: Dict[str, np.ndarray], out_h: int, out_w: int) -> np.ndarray:
+    """Semantic task head on one image: [256, g, g] -> class logits [n_classes, out_h, out_w]."""
+    lat = conv2d(p4, hw["lat_w"], hw["lat_b"], 0)
+    sm = conv2d(lat, hw["smooth_w"], hw["smooth_b"], 1)
+    h = gelu(group_norm(sm, 32, hw["gn_w"], hw["gn_b"]))
+    logits = conv2d(h, hw["pred_w"], hw["pred_b"], 0)
+    return bilinear_resize(logits, out_h, out_w)
+
+
+def dense_head(taps: Dict[int, np.ndarray], head_weights, spec, out_hw: Tuple[int, int]) -> Dict[str, np.ndarray]:
+    """Projector + task head on a batch: taps {l: [B, D, g, g]} (forward's output, four layers of
+    spec.taps in order) -> {"p4": [B, 256, g, g], "logits": [B, n_classes, H, W]}."""
+    hw = {k: ([_to64(t) for t in v] if isinstance(v, (list, tuple)) else _to64(v)) for k, v in head_weights.items()}
+    layers = list(spec.taps)
+    B = taps[layers[0]].shape[0]
+    p4, logits = [], []
+    for i in range(B):
+        p = dense_projector([taps[l][i] for l in layers], hw)
+        p4.append(p)
+        logits.append(dense_task_head(p, hw, out_hw[0], out_hw[1]))
+    return {"p4": np.stack(p4), "logits": np.stack(logits)}
+
+
+def _to64(t) -> np.ndarray:
+    if isinstance(t, np.ndarray):
+        return t.astype(np.float64)
+    return t.detach().double().cpu().numpy()
+

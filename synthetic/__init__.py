@@ -90,10 +90,11 @@ VITG14_224 = ModelSpec("vitg14_224", 14, 224, 224, 1536, 40, 24, 6144, 0, True)
 # Small shapes for fast parity runs (several GEMM tiles and a ragged tail, seconds in fp64).
 TINY_S16 = ModelSpec("tiny_s16", 16, 96, 160, 128, 2, 2, 512, 4, False)            # T = 65
 TINY_S14 = ModelSpec("tiny_s14", 14, 126, 126, 128, 3, 2, 256, 0, True, (1, 3))     # T = 82
+TINY_S14_DENSE = ModelSpec("tiny_s14_dense", 14, 126, 126, 128, 4, 2, 256, 0, True, (1, 2, 3, 4))  # four taps
 SMALL_S16 = ModelSpec("small_s16", 16, 224, 224, 256, 3, 4, 1024, 4, False, (2,))   # T = 201
 
 PRESETS: Dict[str, ModelSpec] = {
-    s.name: s for s in (VITS16_336, VITS14_518, VITL16_1024, VITL16_384, VITB14_224, VITG14_224, TINY_S16, TINY_S14,
+    s.name: s for s in (VITS16_336, VITS14_518, VITL16_1024, VITL16_384, VITB14_224, VITG14_224, TINY_S16, TINY_S14, TINY_S14_DENSE,
                         SMALL_S16)
 }
 
@@ -202,6 +203,45 @@ def make_head_weights(spec: ModelSpec, seed: int, n_blocks: int = DINOTXT_HEAD_B
         b["qkv_w"] = to_bf16(b["qkv_w"])
         b["qkv_b"] = to_bf16(b["qkv_b"])
     return blocks
+
+
+DENSE_CLASSES = 19       # [diagram] "Predict Conv2d 1x1: 256 to 19 class logits"
+DENSE_WIDTH = 256        # [diagram] "Projector P4": 1,536 to 256
+DENSE_SEED = 5190
+
+
+def make_dense_head_weights(spec: ModelSpec, seed: int, n_classes: int = DENSE_CLASSES,
+                            width: int = DENSE_WIDTH) -> Dict[str, object]:
+    """Seeded bf16 weights of the dense head on the taps (C2f projector P4 + semantic task head),
+    drawn like make_weights: conv weights and biases N(0, 0.02), norm gamma 1 + N(0, 0.02) and
+    beta N(0, 0.02).  Conv weights are [out, in, k, k]; ``bn_w`` lists the six 3x3 convs of the
+    three bottlenecks in order."""
+    g = torch.Generator().manual_seed(int(seed))
+    C4, h = 4 * spec.dim, width // 2
+
+    def ln(n):
+        return to_bf16(1.0 + _normal(g, (n,), 0.02)), to_bf16(_normal(g, (n,), 0.02))
+
+    w: Dict[str, object] = {}
+    w["cv1_w"] = to_bf16(_normal(g, (width, C4, 1, 1), 0.02))
+    w["cv1_ln_w"], w["cv1_ln_b"] = ln(width)
+    w["bn_w"], w["bn_ln_w"], w["bn_ln_b"] = [], [], []
+    for _ in range(6):
+        w["bn_w"].append(to_bf16(_normal(g, (h, h, 3, 3), 0.02)))
+        a, b = ln(h)
+        w["bn_ln_w"].append(a)
+        w["bn_ln_b"].append(b)
+    w["cv2_w"] = to_bf16(_normal(g, (width, 5 * h, 1, 1), 0.02))
+    w["cv2_ln_w"], w["cv2_ln_b"] = ln(width)
+    w["out_ln_w"], w["out_ln_b"] = ln(width)
+    w["lat_w"] = to_bf16(_normal(g, (width, width, 1, 1), 0.02))
+    w["lat_b"] = to_bf16(_normal(g, (width,), 0.02))
+    w["smooth_w"] = to_bf16(_normal(g, (width, width, 3, 3), 0.02))
+    w["smooth_b"] = to_bf16(_normal(g, (width,), 0.02))
+    w["gn_w"], w["gn_b"] = ln(width)
+    w["pred_w"] = to_bf16(_normal(g, (n_classes, width, 1, 1), 0.02))
+    w["pred_b"] = to_bf16(_normal(g, (n_classes,), 0.02))
+    return w
 
 
 # Attention-sink construction (kornia/dinov3 card, "Build BF16, not FP16": the scaled logits

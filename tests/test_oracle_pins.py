@@ -473,6 +473,100 @@ def test_seg_whole_with_head_uses_head_tokens():
     assert _close(scores, up, 1e-10) and np.array_equal(labels, up.argmax(0))
 
 
+# ------------------------------------------------------------------ dense head on the taps
+def torch_dense_head(taps, hw, layers, out_hw):
+    """The projector and task head with torch fp64 ops (F.conv2d, F.layer_norm over channels,
+    F.silu, F.group_norm, F.gelu, F.interpolate) -- shares no code with the oracle."""
+    W = {k: ([t.double() for t in v] if isinstance(v, list) else v.double()) for k, v in hw.items()}
+
+    def cln(x, g, b):
+        return F.layer_norm(x.permute(0, 2, 3, 1), (x.shape[1],), g, b, 1e-6).permute(0, 3, 1, 2)
+
+    def cls_(x, w, g, b, pad):
+        return F.silu(cln(F.conv2d(x, w, padding=pad), g, b))
+
+    x = torch.cat([torch.from_numpy(taps[l]) for l in layers], dim=1)
+    y = cls_(x, W["cv1_w"], W["cv1_ln_w"], W["cv1_ln_b"], 0)
+    a, b = y.chunk(2, dim=1)
+    outs, cur = [a, b], b
+    for i in range(3):
+        cur = cls_(cur, W["bn_w"][2 * i], W["bn_ln_w"][2 * i], W["bn_ln_b"][2 * i], 1)
+        cur = cls_(cur, W["bn_w"][2 * i + 1], W["bn_ln_w"][2 * i + 1], W["bn_ln_b"][2 * i + 1], 1)
+        outs.append(cur)
+    z = cls_(torch.cat(outs, dim=1), W["cv2_w"], W["cv2_ln_w"], W["cv2_ln_b"], 0)
+    p4 = cln(z, W["out_ln_w"], W["out_ln_b"])
+    h = F.conv2d(F.conv2d(p4, W["lat_w"], W["lat_b"]), W["smooth_w"], W["smooth_b"], padding=1)
+    h = F.gelu(F.group_norm(h, 32, W["gn_w"], W["gn_b"], 1e-5))
+    logits = F.interpolate(F.conv2d(h, W["pred_w"], W["pred_b"]), size=out_hw, mode="bilinear", align_corners=False)
+    return p4.numpy(), logits.numpy()
+
+
+def test_dense_head_matches_torch_composition():
+    spec = S.PRESETS["tiny_s14_dense"]
+    w = S.make_weights(spec, 51)
+    hw = S.make_dense_head_weights(spec, 52)
+    im = S.make_images(spec, 2, 53)
+    o = O.forward(im, w, spec)
+    layers = list(spec.taps)
+    assert len(layers) == 4
+    out = O.dense_head(o["taps"], hw, spec, (spec.img_h, spec.img_w))
+    p4, logits = torch_dense_head(o["taps"], hw, layers, (spec.img_h, spec.img_w))
+    assert out["logits"].shape == (2, 19, spec.img_h, spec.img_w)
+    assert _close(out["p4"], p4, 1e-10) and _close(out["logits"], logits, 1e-10)
+
+
+def test_conv2d_matches_brute_force_loops():
+    rng = np.random.default_rng(54)
+    x, w, b = rng.standard_normal((3, 5, 4)), rng.standard_normal((2, 3, 3, 3)), rng.standard_normal(2)
+    ref = np.zeros((2, 5, 4))
+    for o in range(2):
+        for y in range(5):
+            for xx in range(4):
+                acc = b[o]
+                for c in range(3):
+                    for ky in range(3):
+                        for kx in range(3):
+                            yy, xs = y + ky - 1, xx + kx - 1
+                            if 0 <= yy < 5 and 0 <= xs < 4:
+                                acc += w[o, c, ky, kx] * x[c, yy, xs]
+                ref[o, y, xx] = acc
+    assert _close(O.conv2d(x, w, b, 1), ref, 1e-12)
+
+
+def test_group_norm_and_channel_ln_special_cases():
+    rng = np.random.default_rng(55)
+    x = rng.standard_normal((8, 3, 5))
+    one = np.ones(8)
+    zero = np.zeros(8)
+    # GroupNorm with one group per channel is instance norm; with one group, LayerNorm over (C, H, W)
+    inst = (x - x.mean(axis=(1, 2), keepdims=True)) / np.sqrt(x.var(axis=(1, 2), keepdims=True) + 1e-5)
+    assert _close(O.group_norm(x, 8, one, zero), inst, 1e-12)
+    whole = (x - x.mean()) / np.sqrt(x.var() + 1e-5)
+    assert _close(O.group_norm(x, 1, one, zero), whole, 1e-12)
+    cl = O.channel_layer_norm(x, one, zero)
+    assert np.abs(cl.mean(axis=0)).max() < 1e-12 and np.abs((cl ** 2).mean(axis=0) - 1).max() < 1e-5
+    assert _close(O.silu(np.array([0.0, 1.0, -2.0])), np.array([0.0, 1 / (1 + np.exp(-1)), -2 / (1 + np.exp(2))]), 1e-15)
+
+
+def test_planted_bottleneck_shortcut_is_caught(monkeypatch):
+    # a residual inside the bottleneck (the C2f variant the diagram rules out) must not pass
+    spec = S.PRESETS["tiny_s14_dense"]
+    w = S.make_weights(spec, 56)
+    hw = S.make_dense_head_weights(spec, 57)
+    o = O.forward(S.make_images(spec, 1, 58), w, spec)
+    p4, _ = torch_dense_head(o["taps"], hw, list(spec.taps), (spec.img_h, spec.img_w))
+    orig = OV._conv_ln_silu
+    calls = {"n": 0}
+
+    def with_shortcut(x, wt, g, b, pad):
+        y = orig(x, wt, g, b, pad)
+        calls["n"] += 1
+        return y + x if (pad == 1 and calls["n"] % 2 == 0) else y
+    monkeypatch.setattr(OV, "_conv_ln_silu", with_shortcut)
+    bad = O.dense_head(o["taps"], hw, spec, (spec.img_h, spec.img_w))["p4"]
+    assert not _close(bad, p4, 1e-6)
+
+
 # ------------------------------------------------------------------ planted mistakes
 def _mut_gelu_tanh(x):
     return 0.5 * x * (1 + np.tanh(math.sqrt(2 / math.pi) * (x + 0.044715 * x ** 3)))
