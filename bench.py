@@ -272,6 +272,54 @@ def secondary_rate(V, name, steps=20, warmup=5):
             "launch": f"CUDA graph of the {launches} kernel launches of one forward"}
 
 
+def secondary_eager(desc, fn, units, steps=10, warmup=3):
+    """images/s of a call through the public binding, timed with CUDA events on the current
+    stream (eager launches; inputs and weights already on the device)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"workload": desc, "images_per_s": units / (ms / 1000.0), "ms_per_step": ms, "launch": "eager"}
+
+
+def secondary_dense(V):
+    """Encoder + dense head on the taps (projector P4 + task head, 19 classes at 518 x 518)."""
+    spec, w, im = S.make_workload("vits14_518_b8_taps")
+    enc = V.VitEncoder(spec, w, max_batch=im.shape[0])
+    enc.set_dense_head(S.make_dense_head_weights(spec, S.DENSE_SEED))
+    x = im.cuda()
+    r = secondary_eager("ViT-S/14@518, taps 3/6/9/12 + dense head (C2f projector P4, semantic head, 19 classes "
+                        "at 518 x 518), batch 8", lambda: enc.forward_dense(x), x.shape[0])
+    r["launches_per_step"] = enc.last_launch_count()
+    enc.poll()
+    enc.close()
+    return r
+
+
+def secondary_zero_shot(V):
+    """Zero-shot slide scoring of one 512 x 1024 image: 10 ViT-L/16 windows of 384 + the dino.txt
+    vision head + 150 classes."""
+    spec, w, im = S.make_workload("vitl16_slide_512x1024")
+    enc = V.VitEncoder(spec, w, max_batch=10)
+    enc.set_text_head(S.make_head_weights(spec, S.HEAD_SEED))
+    text = S.make_text_feats(S.SLIDE_CLASSES, spec.dim).cuda()
+    x = im[0].cuda()
+    r = secondary_eager("zero-shot slide: one 512 x 1024 image, 10 ViT-L/16 windows of 384 at stride 192, "
+                        "dino.txt head (2 blocks), 150 classes",
+                        lambda: enc.seg(x, text, mode=V.VIT_SEG_SLIDE, side=S.SLIDE_SIDE, stride=S.SLIDE_STRIDE), 1)
+    r["launches_per_step"] = enc.last_launch_count()
+    enc.poll()
+    enc.close()
+    return r
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -351,7 +399,8 @@ def main(argv=None):
     enc.close()
     if rank == 0:
         if not args.no_secondary:
-            line["secondary"] = [secondary_rate(V, "vits16_336_b64_outlier"), secondary_rate(V, "vits16_336_b1")]
+            line["secondary"] = [secondary_rate(V, "vits16_336_b64_outlier"), secondary_rate(V, "vits16_336_b1"),
+                                 secondary_dense(V), secondary_zero_shot(V)]
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl)
         print(json.dumps(line), flush=True)

@@ -173,6 +173,49 @@ vit_status vit_set_text_head(vit_model *m, const vit_block_weights *blocks, int3
 vit_status vit_forward_text_tokens(vit_model *m, const float *images, int32_t B, int32_t H, int32_t W,
                                    float *tokens, void *ws, size_t ws_bytes, vit_stream_t stream);
 
+/* Dense head on the four taps (LibreYOLO DINOv2 configuration diagram: "Projector P4",
+ * "Projector Bottleneck", "Projector output ConvX", "Task head").  bf16 device weights in
+ * PyTorch layouts, borrowed as in vit_create except where noted; W = width, h = W / 2,
+ * D4 = 4 * dim (the four taps concatenated in tap order). */
+typedef struct vit_dense_head_weights {
+  int32_t n_classes;                   /* K: prediction channels (19 in the diagram), 1..1024 */
+  int32_t width;                       /* W: projector width (256 in the diagram); must be 256 */
+  const void *cv1_w;                   /* [W, D4, 1, 1] 1x1 conv, no bias */
+  const void *cv1_ln_w, *cv1_ln_b;     /* [W] channel LayerNorm */
+  const void *bn_w[6];                 /* [h, h, 3, 3] bottleneck convs, no bias: bottleneck i uses 2i, 2i+1 */
+  const void *bn_ln_w[6], *bn_ln_b[6]; /* [h] their channel LayerNorms */
+  const void *cv2_w;                   /* [W, 5h, 1, 1] output ConvX, no bias */
+  const void *cv2_ln_w, *cv2_ln_b;     /* [W] */
+  const void *out_ln_w, *out_ln_b;     /* [W] final channel LayerNorm */
+  const void *lat_w, *lat_b;           /* [W, W, 1, 1], [W] lateral conv */
+  const void *smooth_w, *smooth_b;     /* [W, W, 3, 3], [W] smoothing conv */
+  const void *gn_w, *gn_b;             /* [W] GroupNorm (32 groups) */
+  const void *pred_w, *pred_b;         /* [K, W, 1, 1], [K] prediction conv */
+} vit_dense_head_weights;
+
+/* Attach the dense head (once per model; the model must have exactly four taps in tap_mask).
+ * Makes the 3x3 weights' GEMM copies and fp32 copies of the vectors and of pred_w now; cv1_w,
+ * cv2_w and lat_w are borrowed.  Call with the model's device current.
+ * Projector: concat of the four final-norm taps -> 1x1 conv -> channel LN -> SiLU -> split in
+ * halves a, b -> three chained bottlenecks on b (3x3 conv, channel LN, SiLU, twice; no
+ * residual) -> concat a, b, the three bottleneck outputs -> 1x1 conv -> channel LN -> SiLU ->
+ * final channel LN.  Task head: 1x1 lateral conv, 3x3 smoothing conv, GroupNorm(32), GELU,
+ * (dropout: identity), 1x1 prediction conv, bilinear resize (align_corners = false) to H x W.
+ * Channel LN: biased variance, eps 1e-6; GroupNorm eps 1e-5.  Activations between the convs
+ * are bf16 (fp32 accumulation and statistics).  VIT_E_INVALID_ARG / VIT_E_UNSUPPORTED on bad
+ * weights or configuration. */
+vit_status vit_set_dense_head(vit_model *m, const vit_dense_head_weights *w);
+
+/* Workspace of vit_forward_dense for B images of H x W (as vit_forward_hw's sizes). */
+vit_status vit_dense_workspace_size(const vit_model *m, int32_t B, int32_t H, int32_t W, size_t *bytes);
+
+/* Encoder + dense head on B images [B, 3, H, W] (device fp32, normalised):
+ *   logits  device fp32 [B, K, H, W] class logits at the input resolution (required);
+ *   p4      device fp32 [B, W, floor(H/p), floor(W/p)] projector output, or NULL.
+ * Enqueues on `stream`.  VIT_E_INVALID_ARG if no dense head is attached. */
+vit_status vit_forward_dense(vit_model *m, const float *images, int32_t B, int32_t H, int32_t W, float *logits,
+                             float *p4, void *ws, size_t ws_bytes, vit_stream_t stream);
+
 /* Zero-shot dense scoring ([dinotxt] patch/text alignment; whole and slide modes). */
 enum { VIT_SEG_WHOLE = 0, VIT_SEG_SLIDE = 1 };
 
@@ -236,7 +279,7 @@ int32_t vit_last_launch_count(const vit_model *m);
 enum {
   VIT_K_IM2COL = 0, VIT_K_PATCH_GEMM, VIT_K_PREFIX, VIT_K_QKV_GEMM, VIT_K_ATTENTION, VIT_K_PROJ_GEMM,
   VIT_K_FC1_GEMM, VIT_K_FC2_GEMM, VIT_K_TAP, VIT_K_FINAL_LN, VIT_K_SEG_NORM, VIT_K_SEG_COS, VIT_K_SEG_MAP,
-  VIT_K_POS_RESIZE, VIT_K_HEAD_OUT, VIT_K_COUNT
+  VIT_K_POS_RESIZE, VIT_K_HEAD_OUT, VIT_K_DENSE_GEMM, VIT_K_DENSE_AUX, VIT_K_COUNT
 };
 vit_status vit_profile_begin(vit_model *m, int32_t capacity);
 vit_status vit_profile_end(vit_model *m, float *total_ms, int32_t *launches);

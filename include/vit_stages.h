@@ -30,6 +30,11 @@ vit_status vit_stage_linear(const void *A, const void *W, const float *bias, int
 vit_status vit_stage_attention(const void *qkv, int32_t B, int32_t T, int32_t heads, void *out, int32_t *status,
                                vit_stream_t stream);
 
+/* GELU as the FC1 epilogue evaluates it ([diagram] "Encoder block": exact erf form, with erf from
+ * Abramowitz & Stegun 7.1.28, absolute error <= 1.5e-7 |x| plus fp32 rounding):
+ * y[i] = GELU(x[i]) for 0 <= i < n; x, y device fp32.  Enqueues on `stream`. */
+vit_status vit_stage_gelu(const float *x, int64_t n, float *y, vit_stream_t stream);
+
 /* Position-embedding resize ([diagram] "DINOv2-S encoder": "Bicubic interpolation" of the
  * learned grid to the input's patch grid), the kernel vit_forward_hw runs first:
  *   pos: fp32 [(pos_on_cls ? 1 : 0) + gh0 * gw0, D], the patch rows in row-major grid order;

@@ -45,6 +45,8 @@ int main(void) {
   printf("%zu %zu %zu %zu\n", sizeof(vit_config), sizeof(vit_block_weights), sizeof(vit_weights), sizeof(vit_outputs));
   printf("%zu %zu %zu %zu\n", offsetof(vit_config, ln_eps), offsetof(vit_outputs, patch_fp32),
          offsetof(vit_outputs, taps), offsetof(vit_outputs, hidden));
+  printf("%zu %zu %zu %zu\n", sizeof(vit_dense_head_weights), offsetof(vit_dense_head_weights, bn_w),
+         offsetof(vit_dense_head_weights, cv2_w), offsetof(vit_dense_head_weights, pred_b));
   return 0;
 }
 '''
@@ -60,6 +62,9 @@ int main(void) {
                      ctypes.sizeof(V.VitOutputs)]
     assert offs == [V.VitConfig.ln_eps.offset, V.VitOutputs.patch_fp32.offset, V.VitOutputs.taps.offset,
                     V.VitOutputs.hidden.offset]
+    dense = [int(x) for x in lines[2].split()]
+    D = V.VitDenseHeadWeights
+    assert dense == [ctypes.sizeof(D), D.bn_w.offset, D.cv2_w.offset, D.pred_b.offset]
 
 
 def _cfg(**kw):

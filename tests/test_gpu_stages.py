@@ -103,3 +103,24 @@ def test_attention_huge_logits_stay_finite():
     assert np.abs(g - r).max() <= 1e-2 * np.abs(r).max() + 2e-3
     # the sink takes all the weight: every row equals v of key 1
     assert np.abs(g[0] - qkv[0, 1, 2 * D:].double().numpy()).max() < 1e-2
+
+
+def test_gelu_formula_against_exact_erf():
+    """The epilogue's GELU (Abramowitz & Stegun 7.1.28 erf) against the exact erf form in fp64:
+    the formula's error (at most 1.5e-7 |x|) plus single-precision evaluation (one reciprocal,
+    four squarings, the fp32 result) stays within 3e-7 |x| + 5e-7 over [-12, 12]; exact signs
+    and limits far out.  bf16 outputs resolve 3.9e-3 relative, four orders coarser."""
+    need_cuda()
+    import vision_transformer_encoder_fwd_b200 as V
+    x = torch.linspace(-12, 12, 2_000_001, dtype=torch.float32)
+    x = torch.cat([x, torch.tensor([0.0, -0.0, 1e-30, -1e-30, 40.0, -40.0, 3e38, -3e38])])
+    y = V.stage_gelu(x.cuda())
+    torch.cuda.synchronize()
+    xd = x.double().numpy()
+    ref = O.gelu(xd)
+    err = np.abs(y.double().cpu().numpy() - ref)
+    assert np.isfinite(y.cpu().numpy()).all()
+    assert (err <= 3e-7 * np.abs(xd) + 5e-7).all(), err.max()
+    yl, rl = y.cpu().numpy()[-6:], ref[-6:]            # 1e-30, -1e-30, 40, -40, 3e38, -3e38
+    assert yl[2] == 40.0 and yl[3] == 0.0 and yl[4] == np.float32(3e38) and yl[5] == 0.0 and abs(yl[0] - rl[0]) < 1e-37
+

@@ -25,7 +25,7 @@ VIT_E_NONFINITE = 7
 VIT_SEG_WHOLE = 0
 VIT_SEG_SLIDE = 1
 KERNEL_KINDS = ("im2col", "patch_gemm", "prefix", "qkv_gemm", "attention", "proj_gemm", "fc1_gemm", "fc2_gemm",
-                "tap", "final_ln", "seg_norm", "seg_cos", "seg_map", "pos_resize", "head_out")
+                "tap", "final_ln", "seg_norm", "seg_cos", "seg_map", "pos_resize", "head_out", "dense_gemm", "dense_aux")
 
 
 class VitConfig(ctypes.Structure):
@@ -81,6 +81,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "vit_forward_hw": (I32, [P, P, I32, I32, I32, ctypes.POINTER(VitOutputs), P, SZ, P]),
         "vit_set_text_head": (I32, [P, ctypes.POINTER(VitBlockWeights), I32]),
         "vit_forward_text_tokens": (I32, [P, P, I32, I32, I32, P, P, SZ, P]),
+        "vit_set_dense_head": (I32, [P, ctypes.POINTER(VitDenseHeadWeights)]),
+        "vit_dense_workspace_size": (I32, [P, I32, I32, I32, ctypes.POINTER(SZ)]),
+        "vit_forward_dense": (I32, [P, P, I32, I32, I32, P, P, P, SZ, P]),
         "vit_host_workspace_size": (I32, [P, I32, ctypes.POINTER(SZ)]),
         "vit_forward_host": (I32, [P, P, I32, P, P, P, SZ, P]),
         "vit_forward_noalloc": (I32, [P, P, I32, ctypes.POINTER(VitOutputs), P]),
@@ -96,6 +99,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "vit_stage_linear": (I32, [P, P, P, I32, I32, I32, I32, P, P, P]),
         "vit_stage_attention": (I32, [P, I32, I32, I32, P, P, P]),
         "vit_stage_pos_resize": (I32, [P, I32, I32, I32, I32, I32, I32, P, P]),
+        "vit_stage_gelu": (I32, [P, ctypes.c_int64, P, P]),
     }
     for name, (res, args) in sigs.items():
         f = getattr(lib, name)
@@ -129,6 +133,20 @@ def config_from_spec(spec, max_batch: int) -> VitConfig:
         mask |= 1 << (l - 1)
     return VitConfig(spec.patch, spec.img_h, spec.img_w, spec.dim, spec.depth, spec.heads, spec.mlp, spec.registers,
                      1 if spec.pos_on_cls else 0, max_batch, float(spec.ln_eps), mask)
+
+
+_DENSE_VEC_FIELDS = ("cv1_ln_w", "cv1_ln_b", "cv2_ln_w", "cv2_ln_b", "out_ln_w", "out_ln_b", "lat_b", "smooth_b",
+                     "gn_w", "gn_b", "pred_b")
+
+
+class VitDenseHeadWeights(ctypes.Structure):
+    _fields_ = [("n_classes", ctypes.c_int32), ("width", ctypes.c_int32), ("cv1_w", ctypes.c_void_p),
+                ("cv1_ln_w", ctypes.c_void_p), ("cv1_ln_b", ctypes.c_void_p), ("bn_w", ctypes.c_void_p * 6),
+                ("bn_ln_w", ctypes.c_void_p * 6), ("bn_ln_b", ctypes.c_void_p * 6), ("cv2_w", ctypes.c_void_p),
+                ("cv2_ln_w", ctypes.c_void_p), ("cv2_ln_b", ctypes.c_void_p), ("out_ln_w", ctypes.c_void_p),
+                ("out_ln_b", ctypes.c_void_p), ("lat_w", ctypes.c_void_p), ("lat_b", ctypes.c_void_p),
+                ("smooth_w", ctypes.c_void_p), ("smooth_b", ctypes.c_void_p), ("gn_w", ctypes.c_void_p),
+                ("gn_b", ctypes.c_void_p), ("pred_w", ctypes.c_void_p), ("pred_b", ctypes.c_void_p)]
 
 
 class VitEncoder:
@@ -268,6 +286,47 @@ class VitEncoder:
             self.handle, _ptr(images), B, H, W, _ptr(tok), _ptr(wsb), wsb.numel(), _stream_handle(stream)))
         return tok
 
+    # -------------------------------------------------------------- dense head on the taps
+    def set_dense_head(self, hw) -> None:
+        """vit_set_dense_head: hw = dict of bf16 weights as synthetic.make_dense_head_weights gives."""
+        import torch
+
+        def dev(t):
+            return t.to(device=self.device, dtype=torch.bfloat16).contiguous()
+        self.dense_w = {k: ([dev(t) for t in v] if isinstance(v, list) else dev(v)) for k, v in hw.items()}
+        d = self.dense_w
+        st = VitDenseHeadWeights()
+        st.n_classes = int(d["pred_w"].shape[0])
+        st.width = int(d["cv1_w"].shape[0])
+        for k in ("cv1_w", "cv2_w", "lat_w", "smooth_w", "pred_w") + _DENSE_VEC_FIELDS:
+            setattr(st, k, _ptr(d[k]))
+        for i in range(6):
+            st.bn_w[i] = _ptr(d["bn_w"][i])
+            st.bn_ln_w[i] = _ptr(d["bn_ln_w"][i])
+            st.bn_ln_b[i] = _ptr(d["bn_ln_b"][i])
+        self._dense_struct = st
+        with torch.cuda.device(self.device):
+            _check("vit_set_dense_head", self.lib.vit_set_dense_head(self.handle, ctypes.byref(st)))
+
+    def dense_workspace_size(self, B: int, H: int, W: int) -> int:
+        n = ctypes.c_size_t()
+        _check("vit_dense_workspace_size", self.lib.vit_dense_workspace_size(self.handle, B, H, W, ctypes.byref(n)))
+        return n.value
+
+    def forward_dense(self, images, p4=False, stream=None):
+        """vit_forward_dense: class logits [B, K, H, W] (and projector features [B, W, gh, gw])."""
+        import torch
+        B, H, W = images.shape[0], images.shape[-2], images.shape[-1]
+        gh, gw = self.grid((H, W))
+        K, Wd = int(self.dense_w["pred_w"].shape[0]), int(self.dense_w["cv1_w"].shape[0])
+        logits = torch.empty(B, K, H, W, dtype=torch.float32, device=self.device)
+        feats = torch.empty(B, Wd, gh, gw, dtype=torch.float32, device=self.device) if p4 else None
+        wsb = self._workspace(self.dense_workspace_size(B, H, W))
+        _check("vit_forward_dense", self.lib.vit_forward_dense(
+            self.handle, _ptr(images), B, H, W, _ptr(logits), _ptr(feats), _ptr(wsb), wsb.numel(),
+            _stream_handle(stream)))
+        return logits, feats
+
     # -------------------------------------------------------------- zero-shot
     def seg_workspace_size(self, H, W, C, mode, side, stride) -> int:
         n = ctypes.c_size_t()
@@ -354,3 +413,14 @@ def stage_pos_resize(pos, grid0, grid, pos_on_cls: bool, stream=None):
     _check("vit_stage_pos_resize", lib.vit_stage_pos_resize(_ptr(pos), grid0[0], grid0[1], grid[0], grid[1], D,
                                                             1 if pos_on_cls else 0, _ptr(out), _stream_handle(stream)))
     return out
+
+
+def stage_gelu(x, stream=None):
+    """vit_stage_gelu: fp32 device tensor -> GELU(x) as the FC1 epilogue computes it."""
+    import torch
+    lib = load_library()
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    _check("vit_stage_gelu", lib.vit_stage_gelu(_ptr(x), x.numel(), _ptr(y), _stream_handle(stream)))
+    return y
+

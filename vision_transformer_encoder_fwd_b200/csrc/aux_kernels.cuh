@@ -4,6 +4,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "gelu.cuh"
 
 namespace vit {
 
@@ -550,4 +551,15 @@ __global__ void seg_whole_kernel(const float* __restrict__ cosm, int C, int gh, 
   if (labels) labels[pix] = best_c;
 }
 
+// y = GELU(x) elementwise with the epilogues' formula (gelu2), for checking it on its own.
+__global__ void gelu_stage_kernel(const float* __restrict__ x, long long n, float* __restrict__ y) {
+  for (long long i = 2 * (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x); i < n;
+       i += 2LL * gridDim.x * blockDim.x) {
+    const float2 g = gelu2(make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f));
+    y[i] = g.x;
+    if (i + 1 < n) y[i + 1] = g.y;
+  }
+}
+
 }  // namespace vit
+

@@ -20,6 +20,7 @@
 
 #include "cluster.cuh"
 #include "common.cuh"
+#include "gelu.cuh"
 
 namespace vit {
 
@@ -82,35 +83,47 @@ __device__ __forceinline__ void merge_stats(float& n, float& mean, float& m2, fl
   n = tot;
 }
 
-// Affine epilogue of one 32-column chunk for BIAS / LNFOLD: v <- act(rstd * v - rstd * mu * c + b).
+// Affine epilogue of one 32-column chunk for BIAS / LNFOLD: v <- act(rstd * v - rstd * mu * c + b),
+// two columns per packed f32x2 instruction.
 template <int MODE>
 __device__ __forceinline__ void epi_affine(const EpiParams& ep, float (&v)[32], int n, float mu, float rstd) {
   const float4* b4 = reinterpret_cast<const float4*>(ep.bias + n);
   if (MODE == EPI_LNFOLD) {
     const float4* c4 = reinterpret_cast<const float4*>(ep.colsum + n);
-    const float rm = rstd * mu;
+    const float2 nrm = make_float2(-rstd * mu, -rstd * mu);
+    const float2 rs = make_float2(rstd, rstd);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const float4 bb = __ldg(b4 + j);
       const float4 cc = __ldg(c4 + j);
-      v[4 * j + 0] = fmaf(rstd, v[4 * j + 0], fmaf(-rm, cc.x, bb.x));
-      v[4 * j + 1] = fmaf(rstd, v[4 * j + 1], fmaf(-rm, cc.y, bb.y));
-      v[4 * j + 2] = fmaf(rstd, v[4 * j + 2], fmaf(-rm, cc.z, bb.z));
-      v[4 * j + 3] = fmaf(rstd, v[4 * j + 3], fmaf(-rm, cc.w, bb.w));
+      const float2 t0 = ffma2(nrm, make_float2(cc.x, cc.y), make_float2(bb.x, bb.y));
+      const float2 t1 = ffma2(nrm, make_float2(cc.z, cc.w), make_float2(bb.z, bb.w));
+      const float2 r0 = ffma2(rs, make_float2(v[4 * j + 0], v[4 * j + 1]), t0);
+      const float2 r1 = ffma2(rs, make_float2(v[4 * j + 2], v[4 * j + 3]), t1);
+      v[4 * j + 0] = r0.x;
+      v[4 * j + 1] = r0.y;
+      v[4 * j + 2] = r1.x;
+      v[4 * j + 3] = r1.y;
     }
   } else {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const float4 bb = __ldg(b4 + j);
-      v[4 * j + 0] += bb.x;
-      v[4 * j + 1] += bb.y;
-      v[4 * j + 2] += bb.z;
-      v[4 * j + 3] += bb.w;
+      const float2 r0 = fadd2(make_float2(v[4 * j + 0], v[4 * j + 1]), make_float2(bb.x, bb.y));
+      const float2 r1 = fadd2(make_float2(v[4 * j + 2], v[4 * j + 3]), make_float2(bb.z, bb.w));
+      v[4 * j + 0] = r0.x;
+      v[4 * j + 1] = r0.y;
+      v[4 * j + 2] = r1.x;
+      v[4 * j + 3] = r1.y;
     }
   }
   if (ep.gelu) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+    for (int j = 0; j < 16; ++j) {
+      const float2 g = gelu2(make_float2(v[2 * j], v[2 * j + 1]));
+      v[2 * j] = g.x;
+      v[2 * j + 1] = g.y;
+    }
   }
 }
 

@@ -24,6 +24,7 @@
 #include "../../include/vit_stages.h"
 #include "attention.cuh"
 #include "aux_kernels.cuh"
+#include "dense_head.cuh"
 #include "gemm.cuh"
 
 using namespace vit;
@@ -327,6 +328,17 @@ struct vit_model {
   CUtensorMap tm_patch;
   std::vector<BlockW> blocks;
   std::vector<BlockW> head;  // dino.txt vision head blocks (vit_set_text_head), empty if none
+  struct DenseW {
+    bool on = false;
+    int K = 0, W = 0;
+    const __nv_bfloat16 *cv1_w = nullptr, *cv2_w = nullptr, *lat_w = nullptr;  // borrowed [O, C]
+    __nv_bfloat16* bn_wr[6] = {};     // [h, 9h] (owned)
+    __nv_bfloat16* smooth_wr = nullptr;  // [W, 9W] (owned)
+    float *cv1_ln_w = nullptr, *cv1_ln_b = nullptr, *bn_ln_w[6] = {}, *bn_ln_b[6] = {};
+    float *cv2_ln_w = nullptr, *cv2_ln_b = nullptr, *out_ln_w = nullptr, *out_ln_b = nullptr;
+    float *lat_b = nullptr, *smooth_b = nullptr, *gn_w = nullptr, *gn_b = nullptr;
+    float *pred_w = nullptr, *pred_b = nullptr, *zero = nullptr;
+  } dense;  // dense head on the taps (vit_set_dense_head)
   int* d_status = nullptr;
   int last_launches = 0;
   std::vector<void*> allocs;
@@ -517,7 +529,7 @@ struct Scratch {
 // head attached) the dino.txt vision head runs after the backbone and `out->patch_tokens`
 // (fp32) receives its patch rows; the descriptor is not written then.
 vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, const vit_outputs* out, void* ws,
-                       size_t ws_bytes, cudaStream_t s, bool head = false) {
+                       size_t ws_bytes, cudaStream_t s, bool head = false, __nv_bfloat16* tap_rows = nullptr) {
   const vit_config& c = m->cfg;
   vit_status gst = check_geom(m, B, g);
   if (gst != VIT_OK) return gst;
@@ -683,7 +695,15 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
       CK(cudaMemcpyAsync(out->hidden + static_cast<size_t>(l) * M * D, S.x, static_cast<size_t>(M) * D * 4,
                          cudaMemcpyDeviceToDevice, s));
     if (c.tap_mask & (1u << l)) {
-      if (out && out->taps[tap_i]) {
+      if (tap_rows) {
+        // the dense head's input: final-norm tap rows, concatenated in tap order
+        { const int ps_ = prof_open(m, VIT_K_TAP, s);
+        tap_rows_kernel<<<static_cast<int>((static_cast<long long>(B) * P + 7) / 8), 256, 0, s>>>(
+            S.x, m->norm_w, m->norm_b, B, T, R, D, c.ln_eps, tap_rows, 4 * D, tap_i * D);
+        prof_close(m, ps_, s); }
+        CKL();
+        ++launches;
+      } else if (out && out->taps[tap_i]) {
         { const int ps_ = prof_open(m, VIT_K_TAP, s);
         tap_kernel<<<dim3((P + 31) / 32, B), 256, 0, s>>>(S.x, m->norm_w, m->norm_b, T, R, D, c.ln_eps,
                                                             out->taps[tap_i]);
@@ -978,6 +998,274 @@ vit_status vit_forward_text_tokens(vit_model* m, const float* images, int32_t B,
                      /*head=*/true);
 }
 
+// ------------------------------------------------------------------ dense head on the taps
+struct DenseLayout {
+  size_t enc, xc, t, cc, t2, i3, p4, l, stats, lr, total;
+};
+
+static DenseLayout dense_layout(const vit_model* m, int B, const Geom& g) {
+  const size_t Mp = static_cast<size_t>(B) * g.P, D4 = 4 * static_cast<size_t>(m->cfg.dim);
+  const size_t W = m->dense.W, h = W / 2, K = m->dense.K;
+  DenseLayout L;
+  L.enc = ws_layout(m, B, g).total;
+  size_t off = align_up(L.enc, 1024);
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 1024);
+    return at;
+  };
+  L.xc = take(Mp * D4 * 2);
+  L.t = take(Mp * W * 2);
+  L.cc = take(Mp * 5 * h * 2);
+  L.t2 = take(Mp * h * 2);
+  L.i3 = take(Mp * 9 * W * 2);
+  L.p4 = take(Mp * W * 2);
+  L.l = take(Mp * W * 2);
+  L.stats = take(static_cast<size_t>(B) * 32 * 8);
+  L.lr = take(static_cast<size_t>(B) * K * g.P * 4);
+  L.total = off;
+  return L;
+}
+
+static vit_status run_dense(vit_model* m, const float* images, int B, const Geom& g, float* logits, float* p4out,
+                            void* ws, size_t ws_bytes, cudaStream_t s) {
+  const vit_config& c = m->cfg;
+  const auto& dw = m->dense;
+  vit_status st = check_geom(m, B, g);
+  if (st != VIT_OK) return st;
+  const DenseLayout DL = dense_layout(m, B, g);
+  if (!ws || ws_bytes < DL.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) {
+    set_err("dense workspace must be >= %zu bytes and 256-byte aligned", DL.total);
+    return VIT_E_WORKSPACE;
+  }
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(w8 + off); };
+  __nv_bfloat16 *Xc = bf(DL.xc), *Tt = bf(DL.t), *Cc = bf(DL.cc), *T2 = bf(DL.t2), *I3 = bf(DL.i3), *P4 = bf(DL.p4),
+                *Lb = bf(DL.l);
+  float2* gstats = reinterpret_cast<float2*>(w8 + DL.stats);
+  float* lr = reinterpret_cast<float*>(w8 + DL.lr);
+  const int D4 = 4 * c.dim, W = dw.W, h = W / 2, K = dw.K, P = g.P;
+  const long long Mp = static_cast<long long>(B) * P;
+
+  ImgSrc src{images, 3LL * g.H * g.W, static_cast<long long>(g.H) * g.W, g.W, 1, 0, 0, 0};
+  vit_outputs none{};
+  st = run_forward(m, src, B, g, &none, ws, DL.enc, s, false, Xc);
+  if (st != VIT_OK) return st;
+  int launches = m->last_launches;
+
+  auto gemm = [&](const __nv_bfloat16* A, int lda, int Kd, const __nv_bfloat16* Wt, int N, const float* bias,
+                  __nv_bfloat16* out) -> vit_status {
+    const int bn = pick_bn(static_cast<int>(Mp), N, m->nsm);
+    CUtensorMap ta, tb, to;
+    if (!tmap_2d(&ta, A, Kd, Mp, lda, 64, GEMM_BM) || !tmap_2d(&tb, Wt, Kd, N, Kd, 64, bn == BN_PAIR ? 128 : bn) ||
+        !tmap_out_bf16(&to, out, N, Mp, N))
+      return VIT_E_CUDA;
+    EpiParams ep{};
+    ep.M = static_cast<int>(Mp);
+    ep.N = N;
+    ep.bias = bias;
+    ep.ldo = N;
+    { const int ps_ = prof_open(m, VIT_K_DENSE_GEMM, s);
+    CK(launch_gemm(bn, EPI_BIAS, ta, tb, to, to, static_cast<int>(Mp), N, Kd, ep, m->d_status, s, m->nsm));
+    prof_close(m, ps_, s); }
+    ++launches;
+    return VIT_OK;
+  };
+  const int rows_grid = static_cast<int>((Mp + 7) / 8);
+  auto ln_silu = [&](const __nv_bfloat16* in, int C, const float* lg, const float* lb, const float* lg2,
+                     const float* lb2, int mode, __nv_bfloat16* out, int ld_out, int col0) -> vit_status {
+    { const int ps_ = prof_open(m, VIT_K_DENSE_AUX, s);
+    row_ln_silu_kernel<<<rows_grid, 256, 0, s>>>(in, C, Mp, C, lg, lb, lg2, lb2, 1e-6f, mode, out, ld_out, col0);
+    prof_close(m, ps_, s); }
+    CKL();
+    ++launches;
+    return VIT_OK;
+  };
+  auto im2col = [&](const __nv_bfloat16* in, int ld_in, int col0, int C) -> vit_status {
+    { const int ps_ = prof_open(m, VIT_K_DENSE_AUX, s);
+    im2col3x3_kernel<<<grid_1d(Mp * 9 * (C / 8), 256, m->nsm), 256, 0, s>>>(in, ld_in, col0, C, B, g.gh, g.gw, I3);
+    prof_close(m, ps_, s); }
+    CKL();
+    ++launches;
+    return VIT_OK;
+  };
+#define DENSE_STEP(x)            \
+  do {                           \
+    const vit_status e_ = (x);   \
+    if (e_ != VIT_OK) return e_; \
+  } while (0)
+  // projector P4
+  DENSE_STEP(gemm(Xc, D4, D4, dw.cv1_w, W, dw.zero, Tt));
+  DENSE_STEP(ln_silu(Tt, W, dw.cv1_ln_w, dw.cv1_ln_b, nullptr, nullptr, 0, Cc, 5 * h, 0));
+  for (int i = 0; i < 3; ++i) {
+    const int in_col = (i == 0) ? h : 2 * h + (i - 1) * h;
+    DENSE_STEP(im2col(Cc, 5 * h, in_col, h));
+    DENSE_STEP(gemm(I3, 9 * h, 9 * h, dw.bn_wr[2 * i], h, dw.zero, Tt));
+    DENSE_STEP(ln_silu(Tt, h, dw.bn_ln_w[2 * i], dw.bn_ln_b[2 * i], nullptr, nullptr, 0, T2, h, 0));
+    DENSE_STEP(im2col(T2, h, 0, h));
+    DENSE_STEP(gemm(I3, 9 * h, 9 * h, dw.bn_wr[2 * i + 1], h, dw.zero, Tt));
+    DENSE_STEP(ln_silu(Tt, h, dw.bn_ln_w[2 * i + 1], dw.bn_ln_b[2 * i + 1], nullptr, nullptr, 0, Cc, 5 * h,
+                       2 * h + i * h));
+  }
+  DENSE_STEP(gemm(Cc, 5 * h, 5 * h, dw.cv2_w, W, dw.zero, Tt));
+  DENSE_STEP(ln_silu(Tt, W, dw.cv2_ln_w, dw.cv2_ln_b, dw.out_ln_w, dw.out_ln_b, 1, P4, W, 0));
+  if (p4out) {
+    { const int ps_ = prof_open(m, VIT_K_DENSE_AUX, s);
+    rows_to_chw_kernel<<<grid_1d(Mp * W, 256, m->nsm), 256, 0, s>>>(P4, B, P, W, p4out);
+    prof_close(m, ps_, s); }
+    CKL();
+    ++launches;
+  }
+  // task head
+  DENSE_STEP(gemm(P4, W, W, dw.lat_w, W, dw.lat_b, Lb));
+  DENSE_STEP(im2col(Lb, W, 0, W));
+  DENSE_STEP(gemm(I3, 9 * W, 9 * W, dw.smooth_wr, W, dw.smooth_b, Tt));
+#undef DENSE_STEP
+  { const int ps_ = prof_open(m, VIT_K_DENSE_AUX, s);
+  group_norm_stats_kernel<<<dim3(32, B), 256, 0, s>>>(Tt, P, W, 32, gstats);
+  prof_close(m, ps_, s); }
+  CKL();
+  { const int ps_ = prof_open(m, VIT_K_DENSE_AUX, s);
+  group_norm_gelu_kernel<<<grid_1d(Mp * W / 2, 256, m->nsm), 256, 0, s>>>(Tt, Mp, P, W, 32, gstats, dw.gn_w, dw.gn_b,
+                                                                         1e-5f, Lb);
+  prof_close(m, ps_, s); }
+  CKL();
+  { const int ps_ = prof_open(m, VIT_K_DENSE_AUX, s);
+  predict_kernel<<<rows_grid, 256, 0, s>>>(Lb, Mp, P, W, dw.pred_w, dw.pred_b, K, lr);
+  prof_close(m, ps_, s); }
+  CKL();
+  { const int ps_ = prof_open(m, VIT_K_DENSE_AUX, s);
+  resize_logits_kernel<<<grid_1d(static_cast<long long>(B) * g.H * g.W, 256, m->nsm), 256, 0, s>>>(
+      lr, B, K, g.gh, g.gw, g.H, g.W, logits);
+  prof_close(m, ps_, s); }
+  CKL();
+  launches += 4;
+  m->last_launches = launches;
+  return VIT_OK;
+}
+
+vit_status vit_set_dense_head(vit_model* m, const vit_dense_head_weights* w) {
+  if (!m || !w) {
+    set_err("NULL argument");
+    return VIT_E_INVALID_ARG;
+  }
+  if (m->dense.on) {
+    set_err("a dense head is already attached to this model");
+    return VIT_E_INVALID_ARG;
+  }
+  if (__builtin_popcount(m->cfg.tap_mask) != 4) {
+    set_err("the dense head needs exactly four taps (tap_mask has %d)", __builtin_popcount(m->cfg.tap_mask));
+    return VIT_E_UNSUPPORTED;
+  }
+  if (w->width != 256 || w->n_classes < 1 || w->n_classes > 1024) {
+    set_err("dense head: width must be 256 and n_classes 1..1024 (got %d, %d)", w->width, w->n_classes);
+    return VIT_E_UNSUPPORTED;
+  }
+  const void* ptrs[] = {w->cv1_w, w->cv1_ln_w, w->cv1_ln_b, w->cv2_w, w->cv2_ln_w, w->cv2_ln_b, w->out_ln_w,
+                        w->out_ln_b, w->lat_w, w->lat_b, w->smooth_w, w->smooth_b, w->gn_w, w->gn_b, w->pred_w,
+                        w->pred_b};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) {
+      set_err("dense head: weight pointer NULL or not 16-byte aligned");
+      return VIT_E_INVALID_ARG;
+    }
+  for (int i = 0; i < 6; ++i)
+    if (!w->bn_w[i] || !w->bn_ln_w[i] || !w->bn_ln_b[i] || !aligned16(w->bn_w[i])) {
+      set_err("dense head: bottleneck %d weight pointer NULL or not 16-byte aligned", i);
+      return VIT_E_INVALID_ARG;
+    }
+  int cur = 0;
+  CK(cudaGetDevice(&cur));
+  if (cur != m->device) {
+    set_err("vit_set_dense_head called with device %d current; the model lives on device %d", cur, m->device);
+    return VIT_E_INVALID_ARG;
+  }
+  const int W = w->width, h = W / 2, K = w->n_classes;
+  auto& d = m->dense;
+  cudaStream_t s;
+  CK(cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking));
+  auto run = [&]() -> vit_status {
+    vit_status e;
+    for (int i = 0; i < 6; ++i) {
+      if ((e = alloc_dev(m, reinterpret_cast<void**>(&d.bn_wr[i]), static_cast<size_t>(h) * 9 * h * 2)) != VIT_OK)
+        return e;
+      conv3x3_weight_kernel<<<grid_1d(static_cast<long long>(h) * 9 * h, 256, m->nsm), 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(w->bn_w[i]), h, h, d.bn_wr[i]);
+      CKL();
+      if ((e = to_f32(m, w->bn_ln_w[i], h, &d.bn_ln_w[i], s)) != VIT_OK) return e;
+      if ((e = to_f32(m, w->bn_ln_b[i], h, &d.bn_ln_b[i], s)) != VIT_OK) return e;
+    }
+    if ((e = alloc_dev(m, reinterpret_cast<void**>(&d.smooth_wr), static_cast<size_t>(W) * 9 * W * 2)) != VIT_OK)
+      return e;
+    conv3x3_weight_kernel<<<grid_1d(static_cast<long long>(W) * 9 * W, 256, m->nsm), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(w->smooth_w), W, W, d.smooth_wr);
+    CKL();
+    if ((e = to_f32(m, w->cv1_ln_w, W, &d.cv1_ln_w, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->cv1_ln_b, W, &d.cv1_ln_b, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->cv2_ln_w, W, &d.cv2_ln_w, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->cv2_ln_b, W, &d.cv2_ln_b, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->out_ln_w, W, &d.out_ln_w, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->out_ln_b, W, &d.out_ln_b, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->lat_b, W, &d.lat_b, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->smooth_b, W, &d.smooth_b, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->gn_w, W, &d.gn_w, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->gn_b, W, &d.gn_b, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->pred_w, static_cast<size_t>(K) * W, &d.pred_w, s)) != VIT_OK) return e;
+    if ((e = to_f32(m, w->pred_b, K, &d.pred_b, s)) != VIT_OK) return e;
+    if ((e = alloc_dev(m, reinterpret_cast<void**>(&d.zero), static_cast<size_t>(W) * 4)) != VIT_OK) return e;
+    CK(cudaMemsetAsync(d.zero, 0, static_cast<size_t>(W) * 4, s));
+    CK(cudaStreamSynchronize(s));
+    return VIT_OK;
+  };
+  const vit_status st = run();
+  cudaStreamDestroy(s);
+  if (st != VIT_OK) return st;
+  d.cv1_w = static_cast<const __nv_bfloat16*>(w->cv1_w);
+  d.cv2_w = static_cast<const __nv_bfloat16*>(w->cv2_w);
+  d.lat_w = static_cast<const __nv_bfloat16*>(w->lat_w);
+  d.K = K;
+  d.W = W;
+  d.on = true;
+  return VIT_OK;
+}
+
+vit_status vit_dense_workspace_size(const vit_model* m, int32_t B, int32_t H, int32_t W, size_t* bytes) {
+  if (!m || !bytes) {
+    set_err("NULL argument");
+    return VIT_E_INVALID_ARG;
+  }
+  if (!m->dense.on) {
+    set_err("no dense head attached (vit_set_dense_head)");
+    return VIT_E_INVALID_ARG;
+  }
+  if (B < 1 || B > m->cfg.max_batch) {
+    set_err("batch %d outside 1..max_batch (%d)", B, m->cfg.max_batch);
+    return VIT_E_SHAPE;
+  }
+  const Geom g = geom_for(m, H, W);
+  vit_status st = check_geom(m, B, g);
+  if (st != VIT_OK) return st;
+  *bytes = dense_layout(m, B, g).total;
+  return VIT_OK;
+}
+
+vit_status vit_forward_dense(vit_model* m, const float* images, int32_t B, int32_t H, int32_t W, float* logits,
+                             float* p4, void* ws, size_t ws_bytes, vit_stream_t stream) {
+  if (!m || !images || !logits || !aligned16(images) || !aligned16(logits) || !aligned16(p4)) {
+    set_err("model, images or logits NULL / a pointer not 16-byte aligned");
+    return VIT_E_INVALID_ARG;
+  }
+  if (!m->dense.on) {
+    set_err("no dense head attached (vit_set_dense_head)");
+    return VIT_E_INVALID_ARG;
+  }
+  if (B < 1 || B > m->cfg.max_batch) {
+    set_err("batch %d outside 1..max_batch (%d)", B, m->cfg.max_batch);
+    return VIT_E_SHAPE;
+  }
+  return run_dense(m, images, B, geom_for(m, H, W), logits, p4, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
 vit_status vit_host_workspace_size(const vit_model* m, int32_t batch, size_t* bytes) {
   size_t fw = 0;
   vit_status st = vit_workspace_size(m, batch, &fw);
@@ -1253,6 +1541,20 @@ vit_status vit_stage_attention(const void* qkv, int32_t B, int32_t T, int32_t he
   if (!tmap_qkv3d(&tm, qkv, B, T, heads * 64)) return VIT_E_CUDA;
   CK(launch_attention(tm, static_cast<const __nv_bfloat16*>(qkv), B, T, heads, static_cast<__nv_bfloat16*>(out), status,
                       reinterpret_cast<cudaStream_t>(stream)));
+  return VIT_OK;
+}
+
+vit_status vit_stage_gelu(const float* x, int64_t n, float* y, vit_stream_t stream) {
+  if (!x || !y || n < 0) {
+    set_err("NULL pointer or negative n");
+    return VIT_E_INVALID_ARG;
+  }
+  if (n == 0) return VIT_OK;
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  gelu_stage_kernel<<<grid_1d((n + 1) / 2, 256, device_sms(dev)), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      x, static_cast<long long>(n), y);
+  CKL();
   return VIT_OK;
 }
 
