@@ -375,13 +375,17 @@ def main(argv=None):
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     e0.record(stream)
     for i in range(args.steps):
+        marks[i].record(stream)
         enc.forward_into(imgs[i % 2], outs)
+    marks[args.steps].record(stream)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
+    step_ms = sorted(marks[i].elapsed_time(marks[i + 1]) for i in range(args.steps))
     prof = enc.profile_end()
     enc.poll()
     ms_total = allreduce_max(e0.elapsed_time(e1), dist, "cuda")
@@ -396,6 +400,9 @@ def main(argv=None):
     line = None
     if rank == 0:
         line = report(args, spec, wl, B, world, prof, ms_total, value, e2e, launches_per_step, clk, peaks, imgs, enc)
+        line["step_ms"] = {"median": statistics.median(step_ms),
+                           "p90": step_ms[min(len(step_ms) - 1, int(0.9 * len(step_ms)))],
+                           "min": step_ms[0], "max": step_ms[-1], "rank": "0 (per-step CUDA events)"}
     enc.close()
     if rank == 0:
         if not args.no_secondary:
