@@ -139,8 +139,8 @@ __device__ __forceinline__ void softmax_block_p(const float (&s)[128], float mc,
 }
 
 __global__ void __launch_bounds__(ATT_THREADS, 1)
-    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __nv_bfloat16* __restrict__ qkv, int nimg,
-                       int T, int D, __nv_bfloat16* __restrict__ out, int* gstatus) {
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __nv_bfloat16* __restrict__ qkv, int T, int D,
+                       __nv_bfloat16* __restrict__ out, int* gstatus) {
   extern __shared__ __align__(1024) uint8_t smem[];
   // The swizzled layouts assume 1024-byte aligned tiles; report and stop if the shared window
   // is not (uniform across the CTA, before anything is allocated).
@@ -163,27 +163,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // CTA order (1-D grid): first every full pair of query tiles, pair index fastest so that the
-  // CTAs of one (image, head) run together and share its K/V in L2; then, when the tile count
-  // is odd, the single last tiles, which do half the work and so fill the final wave.
   const int n_qtiles = (T + ATT_BM - 1) / ATT_BM;
-  const int heads = D / 64;
-  const int npairs = n_qtiles / 2;
-  const int nfull = npairs * heads * nimg;  // the host keeps the grid below 2^31
-  const int bx = static_cast<int>(blockIdx.x);
-  int tile0, h, b;
-  if (bx < nfull) {
-    const int hb = bx / npairs;
-    tile0 = 2 * (bx - hb * npairs);
-    h = hb % heads;
-    b = hb / heads;
-  } else {
-    const int hb = bx - nfull;
-    tile0 = n_qtiles - 1;
-    h = hb % heads;
-    b = hb / heads;
-  }
+  const int tile0 = blockIdx.x * 2;
   const int ntile = min(2, n_qtiles - tile0);
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
   const int nkv = (T + ATT_BN - 1) / ATT_BN;
 
   if (threadIdx.x == 0) {

@@ -270,10 +270,8 @@ cudaError_t launch_attention(const CUtensorMap& tm, const __nv_bfloat16* qkv, in
   cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel, AttnCfg::SMEM_BYTES, attr_done);
   if (e != cudaSuccess) return e;
   const int n_qtiles = (T + ATT_BM - 1) / ATT_BM;
-  const long long ctas = static_cast<long long>((n_qtiles + 1) / 2) * heads * B;
-  if (ctas > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  attn_fwd_tc_kernel<<<static_cast<unsigned>(ctas), ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, qkv, B, T, heads * 64,
-                                                                                           out, st);
+  dim3 grid((n_qtiles + 1) / 2, heads, B);
+  attn_fwd_tc_kernel<<<grid, ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, qkv, T, heads * 64, out, st);
   return cudaGetLastError();
 }
 
