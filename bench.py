@@ -151,7 +151,7 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sm, mx, reasons = [], None, set()
+        sm, pw, mx, reasons = [], [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [x.strip() for x in ln.split(",")]
@@ -162,11 +162,15 @@ class ClockSampler:
                 mx = float(parts[2])
             except ValueError:
                 continue
+            try:
+                pw.append(float(parts[3]))
+            except ValueError:
+                pass
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "power_w": statistics.median(pw) if pw else None, "samples": len(sm)}
 
 
 def oracle_sample(spec, weights, images, blocks):
@@ -418,27 +422,38 @@ def main(argv=None):
 
 
 def end_to_end(enc, imgs, spec, B, args, stream, barrier, dist, world):
+    """The same metric through vit_forward_host (pinned host images in; descriptor and bf16 patch
+    tokens back to pinned host memory), copies inside the timed region.  Steps alternate between
+    two streams, each with its own workspace and host output buffers, as a caller pipelining
+    batches would: one step's copies run under the other's kernels."""
     host_imgs = [im.cpu().pin_memory() for im in imgs]
-    desc_h = torch.empty(B, spec.dim, dtype=torch.float32).pin_memory()
-    patch_h = torch.empty(B, spec.n_patches, spec.dim, dtype=torch.bfloat16).pin_memory()
-    hws = torch.empty(enc.host_workspace_size(B), dtype=torch.uint8, device="cuda")
+    desc_h = [torch.empty(B, spec.dim, dtype=torch.float32).pin_memory() for _ in range(2)]
+    patch_h = [torch.empty(B, spec.n_patches, spec.dim, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    hws = [torch.empty(enc.host_workspace_size(B), dtype=torch.uint8, device="cuda") for _ in range(2)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
     for i in range(args.warmup):
-        enc.forward_host(host_imgs[i % 2], desc_h, patch_h, ws=hws)
+        enc.forward_host(host_imgs[i % 2], desc_h[i % 2], patch_h[i % 2], stream=streams[i % 2], ws=hws[i % 2])
     torch.cuda.synchronize()
     barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
+    for st in streams:
+        st.wait_event(f0)
     for i in range(args.steps):
-        enc.forward_host(host_imgs[i % 2], desc_h, patch_h, ws=hws)
+        enc.forward_host(host_imgs[i % 2], desc_h[i % 2], patch_h[i % 2], stream=streams[i % 2], ws=hws[i % 2])
+    for st in streams:
+        stream.wait_stream(st)
     f1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    enc.poll()
+    enc.poll(streams[0])
+    enc.poll(streams[1])
     e2e_value = images_per_s(world, B, args.steps, allreduce_max(f0.elapsed_time(f1), dist, "cuda"))
     h2d = host_imgs[0].numel() * 4
-    d2h = desc_h.numel() * 4 + patch_h.numel() * 2
+    d2h = desc_h[0].numel() * 4 + patch_h[0].numel() * 2
 
-    return {"value": e2e_value, "unit": "images/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    return {"value": e2e_value, "unit": "images/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "streams": 2}
 
 
 def report(args, spec, wl, B, world, prof, ms_total, value, e2e, launches_per_step, clk, peaks, imgs, enc):

@@ -29,6 +29,8 @@ def test_pos_resize_stage(grid0, grid, cls):
 
 
 @pytest.mark.parametrize("name,hw,batch", [("tiny_s16", (128, 128), 2),     # 6x10 grid -> 8x8
+                                           ("tiny_s16", (16, 16), 3),       # one patch: T = 1 + R + 1
+                                           ("tiny_s16", (31, 400), 2),      # 1 x 25 grid, ragged pixels
                                            ("tiny_s14", (98, 154), 3),      # 9x9 -> 7x11
                                            ("tiny_s16", (100, 170), 2),     # floor grid 6x10: the native one
                                            ("small_s16", (288, 160), 2)])   # 14x14 -> 18x10

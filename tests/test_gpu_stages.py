@@ -84,6 +84,31 @@ def test_attention_matches_oracle(B, T, heads, qk_scale):
     assert err <= 1e-2 * np.abs(r).max() + 2e-3, err
 
 
+def test_attention_long_sequence_sampled_rows():
+    """16,389 tokens (ViT-S/16 at 2048 x 2048: 129 key blocks, a ragged last one): sampled query
+    rows of every head against fp64 softmax(q K^T / 8) V computed row by row."""
+    need_cuda()
+    import vision_transformer_encoder_fwd_b200 as V
+    B, T, heads = 1, 16389, 2
+    D = heads * 64
+    qkv = S.make_matrix((B, T, 3 * D), 2048, 1.0).to(torch.bfloat16)
+    out, st = V.stage_attention(qkv.cuda(), heads)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    g = out.double().cpu().numpy()[0]
+    x = qkv.double().numpy()[0]
+    rows = np.random.default_rng(7).choice(T, 48, replace=False).tolist() + [0, 127, 128, T - 5, T - 1]
+    for h in range(heads):
+        k = x[:, D + 64 * h:D + 64 * (h + 1)]
+        v = x[:, 2 * D + 64 * h:2 * D + 64 * (h + 1)]
+        for t in rows:
+            q = x[t, 64 * h:64 * (h + 1)]
+            a = O.attention_probs(q[None], k)[0]
+            ref = a @ v
+            err = np.abs(g[t, 64 * h:64 * (h + 1)] - ref).max()
+            assert err <= 1e-2 * np.abs(ref).max() + 2e-3, (h, t, err)
+
+
 def test_attention_huge_logits_stay_finite():
     """kornia/dinov3 card, "Build BF16, not FP16": scaled logits of ~2e6 must not overflow."""
     need_cuda()
