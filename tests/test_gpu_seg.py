@@ -84,6 +84,32 @@ def test_seg_slide_small():
     enc.close()
 
 
+@pytest.mark.parametrize("side,stride", [(112, 112), (160, 64), (96, 40), (224, 64), (128, 96)])
+def test_seg_slide_window_overlaps(side, stride):
+    """Window overlaps from none to five per axis (pixels covered by 1 to 12 windows, clamped last
+    windows): the GPU head on the GPU's own window tokens against the oracle's."""
+    need_cuda()
+    import vision_transformer_encoder_fwd_b200 as V
+    spec = S.PRESETS["small_s16"]
+    w = S.make_weights(spec, 75)
+    H, W = 256, 400
+    im = S.make_images(spec, 1, 76, H, W)[0]
+    text = S.make_text_feats(11, spec.dim, 77)
+    nwin = len(O.window_origins(H, side, stride)) * len(O.window_origins(W, side, stride))
+    enc = V.VitEncoder(spec, w, max_batch=nwin)
+    probs, labels = enc.seg(im.cuda(), text.cuda(), mode=V.VIT_SEG_SLIDE, side=side, stride=stride)
+    torch.cuda.synchronize()
+    enc.poll()
+    tok = _gpu_tokens(enc, _crops(im.cuda(), side, stride))
+    g = side // spec.patch
+    hp, hl = O.seg_slide_from_tokens(tok, text.double().numpy(), H, W, side, stride, (g, g))
+    gp = probs.double().cpu().numpy()
+    assert np.abs(gp - hp).max() < 1e-5
+    assert np.abs(gp.sum(0) - 1).max() < 1e-4
+    assert_valid_argmax(labels.cpu().numpy(), hp, 2e-5)
+    enc.close()
+
+
 @pytest.mark.slow
 def test_seg_slide_vitl16_512x1024():
     """The full zero-shot workload: ViT-L/16 on 2 x 5 windows of 384 at stride 192, 150 classes."""
