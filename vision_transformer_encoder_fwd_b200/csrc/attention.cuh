@@ -37,6 +37,7 @@ namespace vit {
 
 constexpr int ATT_BM = 128;
 constexpr int ATT_BN = 128;
+constexpr int ATT_NT = 2;  // query tiles per CTA
 constexpr int ATT_THREADS = 320;
 constexpr int ATT_KV_STAGES = 3;
 

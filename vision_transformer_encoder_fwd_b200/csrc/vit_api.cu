@@ -149,7 +149,7 @@ bool tmap_qkv3d(CUtensorMap* tm, const void* base, int B, int T, int D) {
   }
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(3 * D), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(3 * D) * 2, static_cast<cuuint64_t>(T) * 3 * D * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(ATT_BM), 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(ATT_BN), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -270,7 +270,7 @@ cudaError_t launch_attention(const CUtensorMap& tm, const __nv_bfloat16* qkv, in
   cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel, AttnCfg::SMEM_BYTES, attr_done);
   if (e != cudaSuccess) return e;
   const int n_qtiles = (T + ATT_BM - 1) / ATT_BM;
-  dim3 grid((n_qtiles + 1) / 2, heads, B);
+  dim3 grid((n_qtiles + ATT_NT - 1) / ATT_NT, heads, B);
   attn_fwd_tc_kernel<<<grid, ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, qkv, T, heads * 64, out, st);
   return cudaGetLastError();
 }
