@@ -526,7 +526,151 @@ __global__ void seg_slide_kernel(const float* __restrict__ cosm, int C, int g, i
   if (labels) labels[pix] = best_c;
 }
 
-// Whole mode: scores = bilinear upsample of the cosine map [C, gh, gw] to [C, H, W]; argmax.
+// Slide mode on 16 x 16 pixel tiles: the cosine values of every window covering the tile are
+// first staged in shared memory (for each window the <= 4 x 4 grid cells the tile's pixels
+// interpolate from, all classes), then each thread (pixel) runs the same three passes as
+// seg_slide_kernel -- row maximum, exponential sum, then per class the average over windows of
+// softmax(bilinear(cos)) with the argmax -- reading shared instead of global memory, with the
+// exponential from the special-function unit (__expf: the arguments lie in [-2 max|cos|, 0]).
+// Per-window statistics of each pixel also stay in shared memory.  Limits (the host falls back to
+// seg_slide_kernel beyond them): at most SLIDE_TILE_WIN windows per tile, C <= SLIDE_TILE_C.
+constexpr int SLIDE_TILE = 16;
+constexpr int SLIDE_TILE_WIN = 6;
+constexpr int SLIDE_TILE_C = 160;
+constexpr int SLIDE_TILE_CELLS = 16;  // 4 x 4 grid cells per window
+constexpr int SLIDE_TILE_SMEM =
+    SLIDE_TILE_WIN * SLIDE_TILE_C * SLIDE_TILE_CELLS * 4 + SLIDE_TILE_WIN * SLIDE_TILE * SLIDE_TILE * 8;
+
+__device__ __forceinline__ int slide_first(int lo, int side, int stride, int n) {
+  // first window index whose [origin, origin + side) reaches pixel lo (origins clamped at size - side)
+  return min(n - 1, (lo >= side) ? (lo - side) / stride + 1 : 0);
+}
+
+__global__ void seg_slide_tile_kernel(const float* __restrict__ cosm, int C, int g, int H, int W, int side, int stride,
+                                      int ny, int nx, float* __restrict__ probs, int* __restrict__ labels) {
+  extern __shared__ __align__(16) float sm[];
+  float* scos = sm;                                                     // [win][C][16]
+  float* sstat = sm + SLIDE_TILE_WIN * SLIDE_TILE_C * SLIDE_TILE_CELLS;  // [win][256][2]
+  __shared__ int w_iy[SLIDE_TILE_WIN], w_ix[SLIDE_TILE_WIN], w_r0[SLIDE_TILE_WIN], w_c0[SLIDE_TILE_WIN];
+  __shared__ int n_win;
+  const int ty0 = blockIdx.y * SLIDE_TILE, tx0 = blockIdx.x * SLIDE_TILE;
+  const int ty1 = min(H, ty0 + SLIDE_TILE) - 1, tx1 = min(W, tx0 + SLIDE_TILE) - 1;
+  const int gg = g * g;
+  if (threadIdx.x == 0) {
+    // windows overlapping the tile, and for each the first grid row / column its pixels use
+    int n = 0;
+    const int iy_lo = slide_first(ty0, side, stride, ny), ix_lo = slide_first(tx0, side, stride, nx);
+    for (int iy = iy_lo; iy < ny; ++iy) {
+      const int oy = min(iy * stride, H - side);
+      if (oy > ty1) break;
+      if (oy + side <= ty0) continue;
+      for (int ix = ix_lo; ix < nx; ++ix) {
+        const int ox = min(ix * stride, W - side);
+        if (ox > tx1) break;
+        if (ox + side <= tx0) continue;
+        if (n < SLIDE_TILE_WIN) {
+          w_iy[n] = iy;
+          w_ix[n] = ix;
+          w_r0[n] = bilinear_taps(max(ty0, oy) - oy, g, side).i0;
+          w_c0[n] = bilinear_taps(max(tx0, ox) - ox, g, side).i0;
+        }
+        ++n;
+      }
+    }
+    n_win = n;
+  }
+  __syncthreads();
+  const int nw = min(n_win, SLIDE_TILE_WIN);  // the host only launches tiles with <= SLIDE_TILE_WIN windows
+  // stage the 4 x 4 cells of every window, all classes
+  for (int i = threadIdx.x; i < nw * C * SLIDE_TILE_CELLS; i += blockDim.x) {
+    const int w = i / (C * SLIDE_TILE_CELLS);
+    const int rem = i - w * C * SLIDE_TILE_CELLS;
+    const int c = rem / SLIDE_TILE_CELLS, cell = rem % SLIDE_TILE_CELLS;
+    const int r = min(w_r0[w] + (cell >> 2), g - 1), q = min(w_c0[w] + (cell & 3), g - 1);
+    scos[(w * SLIDE_TILE_C + c) * SLIDE_TILE_CELLS + cell] =
+        __ldg(cosm + static_cast<size_t>(w_iy[w] * nx + w_ix[w]) * C * gg + static_cast<size_t>(c) * gg + r * g + q);
+  }
+  __syncthreads();
+  const int y = ty0 + (threadIdx.x >> 4), x = tx0 + (threadIdx.x & 15);
+  if (y >= H || x >= W) return;
+  // per window: covered?, local tap offsets within the staged 4 x 4 cells, weights
+  auto taps = [&](int w, int& o00, int& d01, int& d10, float& a00, float& a01, float& a10, float& a11) -> bool {
+    const int oy = min(w_iy[w] * stride, H - side), ox = min(w_ix[w] * stride, W - side);
+    if (y < oy || y >= oy + side || x < ox || x >= ox + side) return false;
+    const Taps1D tyy = bilinear_taps(y - oy, g, side);
+    const Taps1D txx = bilinear_taps(x - ox, g, side);
+    o00 = (tyy.i0 - w_r0[w]) * 4 + (txx.i0 - w_c0[w]);
+    d01 = txx.i1 - txx.i0;
+    d10 = (tyy.i1 - tyy.i0) * 4;
+    a00 = (1.f - tyy.w1) * (1.f - txx.w1);
+    a01 = (1.f - tyy.w1) * txx.w1;
+    a10 = tyy.w1 * (1.f - txx.w1);
+    a11 = tyy.w1 * txx.w1;
+    return true;
+  };
+  int covered = 0;
+  for (int w = 0; w < nw; ++w) {
+    int o00, d01, d10;
+    float a00, a01, a10, a11;
+    float m = -INFINITY, inv = 0.f;
+    if (taps(w, o00, d01, d10, a00, a01, a10, a11)) {
+      ++covered;
+      const float* base = scos + w * SLIDE_TILE_C * SLIDE_TILE_CELLS + o00;
+      for (int c = 0; c < C; ++c) {
+        const float* q = base + c * SLIDE_TILE_CELLS;
+        m = fmaxf(m, a00 * q[0] + a01 * q[d01] + a10 * q[d10] + a11 * q[d10 + d01]);
+      }
+      float sum = 0.f;
+      for (int c = 0; c < C; ++c) {
+        const float* q = base + c * SLIDE_TILE_CELLS;
+        sum += __expf(a00 * q[0] + a01 * q[d01] + a10 * q[d10] + a11 * q[d10 + d01] - m);
+      }
+      inv = 1.0f / sum;
+    }
+    sstat[(w * 256 + threadIdx.x) * 2] = m;
+    sstat[(w * 256 + threadIdx.x) * 2 + 1] = inv;
+  }
+  const float inv_count = 1.0f / static_cast<float>(covered);
+  const long long pix = static_cast<long long>(y) * W + x;
+  float best = -INFINITY;
+  int best_c = 0;
+  // classes in groups of 16: the window's taps are computed once per group, the group's partial
+  // averages stay in registers
+  constexpr int CG = 16;
+  for (int c0 = 0; c0 < C; c0 += CG) {
+    float acc[CG];
+#pragma unroll
+    for (int k = 0; k < CG; ++k) acc[k] = 0.f;
+    for (int w = 0; w < nw; ++w) {
+      int o00, d01, d10;
+      float a00, a01, a10, a11;
+      if (!taps(w, o00, d01, d10, a00, a01, a10, a11)) continue;
+      const float m = sstat[(w * 256 + threadIdx.x) * 2], inv = sstat[(w * 256 + threadIdx.x) * 2 + 1];
+      const float* base = scos + (w * SLIDE_TILE_C + c0) * SLIDE_TILE_CELLS + o00;
+#pragma unroll
+      for (int k = 0; k < CG; ++k) {
+        if (c0 + k < C) {
+          const float* q = base + k * SLIDE_TILE_CELLS;
+          const float v = a00 * q[0] + a01 * q[d01] + a10 * q[d10] + a11 * q[d10 + d01];
+          acc[k] += __expf(v - m) * inv;
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < CG; ++k) {
+      if (c0 + k < C) {
+        const float p = acc[k] * inv_count;
+        if (probs) probs[static_cast<size_t>(c0 + k) * H * W + pix] = p;
+        if (p > best) {
+          best = p;
+          best_c = c0 + k;
+        }
+      }
+    }
+  }
+  if (labels) labels[pix] = best_c;
+}
+
 __global__ void seg_whole_kernel(const float* __restrict__ cosm, int C, int gh, int gw, int H, int W,
                                  float* __restrict__ scores, int* __restrict__ labels) {
   const long long pix = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;

@@ -1424,9 +1424,34 @@ vit_status vit_seg_zero_shot(vit_model* m, const float* image, int32_t H, int32_
   launches += 2;
   const long long pix = static_cast<long long>(H) * W;
   if (mode == VIT_SEG_SLIDE) {
+    // the tiled kernel when every 16 x 16 tile meets at most SLIDE_TILE_WIN windows, the classes fit
+    // its shared memory and a grid cell spans at least 8 pixels (a tile then needs <= 4 x 4 cells)
+    auto tile_windows = [&](int size, int n) {
+      int mx = 0;
+      for (int t0 = 0; t0 < size; t0 += SLIDE_TILE) {
+        const int t1 = std::min(size, t0 + SLIDE_TILE) - 1;
+        int cnt = 0;
+        for (int i = 0; i < n; ++i) {
+          const int o = std::min(i * stride, size - side);
+          if (o <= t1 && o + side > t0) ++cnt;
+        }
+        mx = std::max(mx, cnt);
+      }
+      return mx;
+    };
+    const int g = plan.g.gh;
+    const bool tiled = C <= SLIDE_TILE_C && g * 8 <= side && tile_windows(H, ny) * tile_windows(W, nx) <= SLIDE_TILE_WIN;
     { const int ps_ = prof_open(m, VIT_K_SEG_MAP, s);
-    seg_slide_kernel<<<static_cast<int>((pix + 127) / 128), 128, 0, s>>>(cosm, C, plan.g.gh, H, W, side, stride, ny,
-                                                                         nx, probs, labels);
+    if (tiled) {
+      static std::atomic<uint64_t> attr_done{0};
+      CK(set_smem_attr_once(seg_slide_tile_kernel, SLIDE_TILE_SMEM, attr_done));
+      const dim3 grid((W + SLIDE_TILE - 1) / SLIDE_TILE, (H + SLIDE_TILE - 1) / SLIDE_TILE);
+      seg_slide_tile_kernel<<<grid, SLIDE_TILE * SLIDE_TILE, SLIDE_TILE_SMEM, s>>>(cosm, C, g, H, W, side, stride, ny,
+                                                                                    nx, probs, labels);
+    } else {
+      seg_slide_kernel<<<static_cast<int>((pix + 127) / 128), 128, 0, s>>>(cosm, C, g, H, W, side, stride, ny, nx,
+                                                                           probs, labels);
+    }
     prof_close(m, ps_, s); }
   } else {
     { const int ps_ = prof_open(m, VIT_K_SEG_MAP, s);
