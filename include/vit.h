@@ -22,7 +22,9 @@
  *     synchronising (except where stated).  Host validation happens before any launch; on a
  *     validation failure nothing is enqueued.
  *   - Device-side failures (a pipeline wait that ran out of time) set the model's status
- *     word; vit_poll() reads it.  No kernel traps.
+ *     word; vit_poll() reads it.  No kernel traps.  The final LayerNorm (and the dino.txt
+ *     head's) also flags any token row holding a NaN or an infinity; vit_poll() then returns
+ *     VIT_E_NONFINITE.
  */
 #ifndef VIT_B200_H
 #define VIT_B200_H
@@ -44,7 +46,7 @@ typedef enum vit_status {
   VIT_E_WORKSPACE = 4,      /* workspace smaller than vit_*_workspace_size reports */
   VIT_E_CUDA = 5,           /* a CUDA runtime / driver call failed */
   VIT_E_DEVICE_TIMEOUT = 6, /* a device pipeline wait gave up (read via vit_poll) */
-  VIT_E_NONFINITE = 7       /* reserved: non-finite value detected */
+  VIT_E_NONFINITE = 7       /* a NaN or infinity reached the final LayerNorm (read via vit_poll) */
 } vit_status;
 
 /* Encoder architecture.  [diagram] "DINOv2-S encoder" / "Encoder block"; [card] "Model I/O".
@@ -263,8 +265,9 @@ vit_status vit_seg_zero_shot(vit_model *m, const float *image, int32_t H, int32_
 vit_status vit_forward_noalloc(vit_model *m, const float *images, int32_t B, const vit_outputs *out,
                                vit_stream_t stream);
 
-/* Synchronise `stream`, then read and clear the model's device status word.  Returns VIT_OK,
- * VIT_E_DEVICE_TIMEOUT if a kernel gave up on a pipeline wait since the last poll, or
+/* Synchronise `stream`, then read and clear the model's device status words.  Returns VIT_OK,
+ * VIT_E_DEVICE_TIMEOUT if a kernel gave up on a pipeline wait since the last poll,
+ * VIT_E_NONFINITE if a token row reaching the final LayerNorm held a NaN or an infinity, or
  * VIT_E_CUDA if the stream reports an error. */
 vit_status vit_poll(vit_model *m, vit_stream_t stream);
 

@@ -152,3 +152,24 @@ def test_vitb14_224_b64_paired_gemms():
     ref = O.forward(im, w, spec, record_hidden=True, image_indices=keep)
     assert_forward_parity(g, ref, spec, keep)
 
+
+
+def test_nonfinite_input_is_reported_by_poll():
+    """A NaN pixel propagates through the encoder; the final LayerNorm flags the non-finite rows and
+    vit_poll reports VIT_E_NONFINITE once (the flag is cleared by the poll)."""
+    need_cuda()
+    import vision_transformer_encoder_fwd_b200 as V
+    spec = S.PRESETS["tiny_s16"]
+    enc = V.VitEncoder(spec, S.make_weights(spec, 81), max_batch=2)
+    im = S.make_images(spec, 2, 82).cuda()
+    enc.forward(im)
+    enc.poll()                                  # clean input: no error
+    bad = im.clone()
+    bad[1, 0, 5, 7] = float("nan")
+    enc.forward(bad)
+    with pytest.raises(V.VitError) as e:
+        enc.poll()
+    assert e.value.status == V.VIT_E_NONFINITE
+    enc.forward(im)
+    enc.poll()                                  # flag cleared
+    enc.close()

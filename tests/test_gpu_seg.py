@@ -110,6 +110,37 @@ def test_seg_slide_window_overlaps(side, stride):
     enc.close()
 
 
+@pytest.mark.parametrize("C", [1, 160, 161, 300])
+@pytest.mark.parametrize("slide", [False, True])
+def test_seg_class_counts(C, slide):
+    """Class counts from 1 to 300: one and several 64-class tiles of the cosine GEMM, and the tiled
+    slide-scoring kernel's 160-class limit on both sides (beyond it the per-pixel kernel runs),
+    checked against the oracle's head on the GPU's own tokens."""
+    need_cuda()
+    import vision_transformer_encoder_fwd_b200 as V
+    spec = S.PRESETS["small_s16"]
+    w = S.make_weights(spec, 85)
+    H, W, side, stride = (256, 400, 224, 112) if slide else (spec.img_h, spec.img_w, 0, 0)
+    im = S.make_images(spec, 1, 86, H, W)
+    text = S.make_text_feats(C, spec.dim, 87)
+    nwin = len(O.window_origins(H, side, stride)) * len(O.window_origins(W, side, stride)) if slide else 1
+    enc = V.VitEncoder(spec, w, max_batch=nwin)
+    if slide:
+        scores, labels = enc.seg(im[0].cuda(), text.cuda(), mode=V.VIT_SEG_SLIDE, side=side, stride=stride)
+        tok = _gpu_tokens(enc, _crops(im[0].cuda(), side, stride))
+        hs, _ = O.seg_slide_from_tokens(tok, text.double().numpy(), H, W, side, stride,
+                                        (side // spec.patch, side // spec.patch))
+    else:
+        scores, labels = enc.seg(im[0].cuda(), text.cuda(), mode=V.VIT_SEG_WHOLE)
+        tok = _gpu_tokens(enc, im.cuda())
+        hs, _ = O.seg_whole_from_tokens(tok[0], text.double().numpy(), H, W, (spec.grid_h, spec.grid_w))
+    torch.cuda.synchronize()
+    enc.poll()
+    assert np.abs(scores.double().cpu().numpy() - hs).max() < 1e-5
+    assert_valid_argmax(labels.cpu().numpy(), hs, 2e-5)
+    enc.close()
+
+
 @pytest.mark.slow
 def test_seg_slide_vitl16_512x1024():
     """The full zero-shot workload: ViT-L/16 on 2 x 5 windows of 384 at stride 192, 150 classes."""

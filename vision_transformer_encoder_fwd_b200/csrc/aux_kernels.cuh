@@ -169,7 +169,7 @@ __device__ __forceinline__ void row_mean_rstd(const float* __restrict__ xr, int 
 // (image, token) with token 0 (CLS) or 1 + R .. T - 1 (patches).
 __global__ void final_ln_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ be,
                                 int B, int T, int R, int D, float eps, float* __restrict__ desc, void* __restrict__ patch,
-                                int patch_fp32) {
+                                int patch_fp32, int* __restrict__ nonfinite) {
   const int P = T - 1 - R;
   const int warps_per_block = blockDim.x >> 5;
   const long long job = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5);
@@ -182,6 +182,8 @@ __global__ void final_ln_kernel(const float* __restrict__ x, const float* __rest
   const float* xr = x + (static_cast<size_t>(b) * T + t) * D;
   float mean, rstd;
   row_mean_rstd(xr, D, eps, mean, rstd);
+  // a NaN or infinity anywhere in the row reaches its mean or its rstd
+  if (lane == 0 && !(isfinite(mean) && isfinite(rstd))) atomicExch(nonfinite, 1);
   if (j == 0) {
     if (desc == nullptr) return;
     float q = 0.f;
@@ -212,7 +214,8 @@ __global__ void final_ln_kernel(const float* __restrict__ x, const float* __rest
 // group of gcols (64 or 128) columns is kept in registers between its two passes.
 __global__ void final_ln_stream_kernel(float* __restrict__ x, const float* __restrict__ g,
                                        const float* __restrict__ be, long long rows, int D, float eps, int gcols,
-                                       __nv_bfloat16* __restrict__ xb, float2* __restrict__ stats) {
+                                       __nv_bfloat16* __restrict__ xb, float2* __restrict__ stats,
+                                       int* __restrict__ nonfinite) {
   const int warps_per_block = blockDim.x >> 5;
   const long long row = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -220,6 +223,7 @@ __global__ void final_ln_stream_kernel(float* __restrict__ x, const float* __res
   float* xr = x + static_cast<size_t>(row) * D;
   float mean, rstd;
   row_mean_rstd(xr, D, eps, mean, rstd);
+  if (lane == 0 && !(isfinite(mean) && isfinite(rstd))) atomicExch(nonfinite, 1);
   __syncwarp();
   const int per = gcols / 32;  // 2 or 4
   const int ng = D / gcols;

@@ -720,7 +720,7 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
     const long long rows = static_cast<long long>(M);
     { const int ps_ = prof_open(m, VIT_K_FINAL_LN, s);
     final_ln_stream_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(S.x, m->norm_w, m->norm_b, rows, D, c.ln_eps,
-                                                                          m->stats_cols, S.xb, S.stats);
+                                                                          m->stats_cols, S.xb, S.stats, m->d_status + 1);
     prof_close(m, ps_, s); }
     CKL();
     ++launches;
@@ -740,7 +740,8 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
     const long long jobs = static_cast<long long>(B) * (1 + P);
     { const int ps_ = prof_open(m, VIT_K_FINAL_LN, s);
     final_ln_kernel<<<static_cast<int>((jobs + 7) / 8), 256, 0, s>>>(S.x, m->norm_w, m->norm_b, B, T, R, D, c.ln_eps,
-                                                                    out->desc, out->patch_tokens, out->patch_fp32);
+                                                                    out->desc, out->patch_tokens, out->patch_fp32,
+                                                                    m->d_status + 1);
     prof_close(m, ps_, s); }
     CKL();
     ++launches;
@@ -1470,12 +1471,16 @@ vit_status vit_poll(vit_model* m, vit_stream_t stream) {
     return VIT_E_INVALID_ARG;
   }
   CK(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
-  int v = 0;
-  CK(cudaMemcpy(&v, m->d_status, 4, cudaMemcpyDeviceToHost));
-  if (v != 0) {
-    CK(cudaMemset(m->d_status, 0, 4));
-    set_err("a kernel gave up on a pipeline wait (site 0x%x)", v);
+  int v[2] = {0, 0};
+  CK(cudaMemcpy(v, m->d_status, 8, cudaMemcpyDeviceToHost));
+  if (v[0] != 0 || v[1] != 0) CK(cudaMemset(m->d_status, 0, 8));
+  if (v[0] != 0) {
+    set_err("a kernel gave up on a pipeline wait (site 0x%x)", v[0]);
     return VIT_E_DEVICE_TIMEOUT;
+  }
+  if (v[1] != 0) {
+    set_err("a non-finite value reached the final LayerNorm");
+    return VIT_E_NONFINITE;
   }
   return VIT_OK;
 }
