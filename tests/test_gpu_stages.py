@@ -28,6 +28,9 @@ def _ref_linear(A, W, b, gelu):
     (20000, 1024, 1024, False), # paired tiles; last tile: 32 rows on the first CTA, none on the second
     (10184, 3072, 1024, False), # paired tiles; last tile: 256 + 72 rows
     (4096, 768, 3072, False),   # paired tiles, N = 3 x 256, long K
+    (28544, 1152, 384, False),  # ViT-S/16@336 b64 QKV: paired tiles, last column tile padded
+    (10000, 384, 1536, True),   # padded paired tiles, long K, GELU; last row tile: 16 rows
+    (9500, 640, 512, False),    # padded paired tiles, N = 2 x 256 + 128; last row tile: 28 rows
 ])
 def test_linear_matches_oracle(M, N, K, gelu):
     need_cuda()

@@ -51,7 +51,8 @@ struct EpiParams {
   float* x;              // [rows, N] fp32 residual stream (PATCH writes it directly)
   __nv_bfloat16* xb;     // [rows, N] bf16 copy of x (A operand of the next folded GEMM)
   const float* ls;       // [N] layer scale (RESID)
-  float2* stats_out;     // [rows, N / (BN/2)] (mean, M2) over each group of BN/2 columns
+  float2* stats_out;     // [rows, N / stats_cols] (mean, M2) over each group of stats_cols columns
+  int stats_cols;        // RESID: 32 x a power of two, dividing BN/2 (PATCH: always BN/2)
   // PATCH: GEMM row m = b * P + p goes to token row b * T + 1 + R + p, position row p + pos_off
   const float* pos;
   int P, T, R, pos_off;
@@ -127,25 +128,51 @@ __device__ __forceinline__ void epi_affine(const EpiParams& ep, float (&v)[32], 
   }
 }
 
+// LNFOLD: the row's LayerNorm mean and 1 / std, rebuilt from the producer's partial (mean, M2)
+// pairs (merged in column order); the loads go out eight at a time so their latencies overlap.
+__device__ __forceinline__ void lnfold_row_stats(const EpiParams& ep, int row, float& mu, float& rstd) {
+  float n = 0.f, mean = 0.f, m2 = 0.f;
+  const float2* s = ep.stats_in + static_cast<size_t>(row) * ep.nt;
+  for (int t0 = 0; t0 < ep.nt; t0 += 8) {
+    float2 st[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) st[u] = (t0 + u < ep.nt) ? s[t0 + u] : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (t0 + u < ep.nt) merge_stats(n, mean, m2, static_cast<float>(ep.nt_cols), st[u].x, st[u].y);
+  }
+  mu = mean;
+  rstd = rsqrtf(m2 / static_cast<float>(ep.D) + ep.eps);
+}
+
+// Pulls the 128-byte lines of v[n0 .. n0 + cols - 1] (cols a multiple of 32) into L1, so that
+// the epilogue's per-column vectors are L1 hits by the time the accumulator is ready.
+__device__ __forceinline__ void prefetch_cols_l1(const float* v, int n0, int cols) {
+  const int lane = threadIdx.x & 31;
+  if (v != nullptr && lane < cols / 32) asm volatile("prefetch.global.L1 [%0];" ::"l"(v + n0 + lane * 32));
+}
+
+// Work a BIAS / LNFOLD epilogue warp does before it waits for its accumulator: the rows'
+// LayerNorm statistics (LNFOLD) and the columns' bias / colsum lines.  (The same prefetch in the
+// residual epilogue, whose x loads already run a chunk ahead, measured 1-2 % slower.)
+template <int BN, int MODE>
+__device__ __forceinline__ void epilogue_prologue(const EpiParams& ep, int row, int n0, float& mu, float& rstd) {
+  mu = 0.f;
+  rstd = 0.f;
+  if (MODE != EPI_BIAS && MODE != EPI_LNFOLD) return;
+  prefetch_cols_l1(ep.bias, n0, BN / 2);
+  if (MODE == EPI_LNFOLD) prefetch_cols_l1(ep.colsum, n0, BN / 2);
+  if (MODE == EPI_LNFOLD && row < ep.M) lnfold_row_stats(ep, row, mu, rstd);
+}
+
 // BIAS / LNFOLD: one warp's half of a tile (rows row0 .. row0 + 31, columns n0 .. n0 + BN/2 - 1),
 // 64 columns per TMA store from the warp's staging buffer `obuf` (32 rows x 128 bytes, 128B
-// swizzle: 16-byte chunk k of row r sits at chunk k ^ (r % 8)).
+// swizzle: 16-byte chunk k of row r sits at chunk k ^ (r % 8)).  mu / rstd: this thread's row
+// statistics (LNFOLD).
 template <int BN, int MODE>
 __device__ __forceinline__ void epilogue_store_bf16(const EpiParams& ep, const CUtensorMap* tmO, uint32_t taddr,
-                                                    int row0, int n0, uint8_t* obuf) {
+                                                    int row0, int n0, uint8_t* obuf, float mu, float rstd) {
   const int lane = threadIdx.x & 31;
-  const int row = row0 + lane;
-  float mu = 0.f, rstd = 0.f;
-  if (MODE == EPI_LNFOLD && row < ep.M) {
-    float n = 0.f, mean = 0.f, m2 = 0.f;
-    const float2* s = ep.stats_in + static_cast<size_t>(row) * ep.nt;
-    for (int t = 0; t < ep.nt; ++t) {
-      const float2 st = s[t];
-      merge_stats(n, mean, m2, static_cast<float>(ep.nt_cols), st.x, st.y);
-    }
-    mu = mean;
-    rstd = rsqrtf(m2 / static_cast<float>(ep.D) + ep.eps);
-  }
 #pragma unroll 1
   for (int g = 0; g < BN / 128; ++g) {
     if (lane == 0) tma_store_wait_read0();  // the previous store has left the staging buffer
@@ -179,7 +206,7 @@ __device__ __forceinline__ void epilogue_store_bf16(const EpiParams& ep, const C
 // RESID: one warp's half of a tile.  x arrives by TMA into xbuf[c & 1] (32 rows x 128 bytes, 128B
 // swizzle), chunk c + 1 is requested while chunk c is processed; the updated x goes back into the
 // same buffer and, with its bf16 copy (xbbuf: 32 rows x 64 bytes, 64B swizzle), out by TMA stores.
-// Row statistics (mean, M2) of the warp's BN/2 columns are written per row.
+// Row statistics (mean, M2) are written per row for each group of ep.stats_cols columns.
 template <int BN>
 __device__ __forceinline__ void epilogue_resid(const EpiParams& ep, const CUtensorMap* tmX, const CUtensorMap* tmXb,
                                                uint32_t taddr, int row0, int n0, uint8_t* xbuf0, uint8_t* xbbuf,
@@ -254,8 +281,15 @@ __device__ __forceinline__ void epilogue_resid(const EpiParams& ep, const CUtens
       q = fmaf(d, d, q);
     }
     merge_stats(run_n, run_mean, run_m2, 32.f, cm, q);
+    if ((n + 32) % ep.stats_cols == 0) {
+      if (row < ep.M)
+        ep.stats_out[static_cast<size_t>(row) * (ep.N / ep.stats_cols) + (n + 32) / ep.stats_cols - 1] =
+            make_float2(run_mean, run_m2);
+      run_n = 0.f;
+      run_mean = 0.f;
+      run_m2 = 0.f;
+    }
   }
-  if (row < ep.M) ep.stats_out[static_cast<size_t>(row) * (ep.N / HALF) + n0 / HALF] = make_float2(run_mean, run_m2);
 }
 
 // PATCH: rows of the GEMM are scattered to token rows, so this epilogue writes directly.
@@ -475,6 +509,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tma_load_2d(wbuf, &tmO1, n0, row0, &wxfull[0]);
         xpending[0] = true;
       }
+      float mu, rstd;
+      epilogue_prologue<BN, MODE>(ep, row0 + lane, n0, mu, rstd);
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 4)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
@@ -487,7 +523,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       } else if (MODE == EPI_PATCH) {
         epilogue_patch<BN>(ep, taddr, row0 + lane, n0);
       } else {
-        epilogue_store_bf16<BN, MODE>(ep, &tmO1, taddr, row0, n0, wbuf);
+        epilogue_store_bf16<BN, MODE>(ep, &tmO1, taddr, row0, n0, wbuf, mu, rstd);
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -619,7 +655,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   const bool skip = ld_shared_cluster_s32(mapa_shared(smem_u32(const_cast<int*>(abort_flag)), 0)) != 0;
 
   const int num_m = (M + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
-  const int num_n = N / BN;
+  // N a multiple of 128: when N = 256 k + 128 the last column tile is padded, its second half of
+  // B rows is zero-filled by the loads and its second column half is neither computed into an
+  // output nor stored
+  const int num_n = (N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int KB = K / GEMM_BK;
   const int cid = static_cast<int>(blockIdx.x >> 1);
@@ -723,23 +762,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       const int nb = tile - mb * num_n;
       const int row0 = mb * 2 * GEMM_BM + static_cast<int>(rank) * GEMM_BM + q * 32;
       const int n0 = nb * BN + half * (BN / 2);
-      if (MODE == EPI_RESID && lane == 0) {
+      const bool active = n0 < N;  // false for the padding half of a last column tile
+      if (MODE == EPI_RESID && active && lane == 0) {
         tma_store_wait_read0();
         mbar_arrive_expect_tx(&wxfull[0], 4096);
         tma_load_2d(wbuf, &tmO1, n0, row0, &wxfull[0]);
         xpending[0] = true;
       }
+      float mu = 0.f, rstd = 0.f;
+      if (active) epilogue_prologue<BN, MODE>(ep, row0 + lane, n0, mu, rstd);
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 8)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + half * (BN / 2));
       __syncwarp();
-      if (MODE == EPI_RESID) {
+      if (MODE == EPI_RESID && active) {
         epilogue_resid<BN>(ep, &tmO1, &tmO2, taddr, row0, n0, wbuf, wbuf + 8192, wxfull, xph, xpending, abort_flag,
                            gstatus, ok);
         if (!ok) break;
-      } else {
-        epilogue_store_bf16<BN, MODE>(ep, &tmO1, taddr, row0, n0, wbuf);
+      } else if (MODE != EPI_RESID && active) {
+        epilogue_store_bf16<BN, MODE>(ep, &tmO1, taddr, row0, n0, wbuf, mu, rstd);
       }
       tc_fence_before();
       __syncwarp();

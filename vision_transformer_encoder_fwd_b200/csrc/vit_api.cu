@@ -228,7 +228,7 @@ cudaError_t launch_gemm_pair_t(const CUtensorMap& a, const CUtensorMap& b, const
     mc = std::max(1, std::min(n, nsm / 2));
     max_clusters.store(mc);
   }
-  const int tiles = ((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * (N / 256);
+  const int tiles = ((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * ((N + 255) / 256);
   const int clusters = std::max(1, std::min(tiles, mc));
   gemm_pair_kernel<MODE><<<2 * clusters, GEMM_THREADS, smem, s>>>(a, b, o1, o2, M, N, K, ep, st);
   return cudaGetLastError();
@@ -280,18 +280,22 @@ int grid_1d(long long work, int block, int nsm) {
   return static_cast<int>(std::max(1LL, std::min(g, static_cast<long long>(nsm) * 32)));
 }
 
-// GEMM tiling: the paired 256 x 256 tile when N allows it and the pairs still fill the SMs,
-// else 128 x 256 per CTA when that fills them, else 128 x 128.
+// GEMM tiling: the paired 256 x 256 tile when the pairs fill the SMs (N = 256 k + 128 pads the
+// last column tile: a tile of 256 x 256 per SM pair moves as many bytes through each SM's shared
+// memory per k-step as one of 128 x 128 per SM, for twice the MMA work), else 128 x 256 per CTA
+// when N allows it and that fills the SMs, else 128 x 128.
 int pick_bn(int M, int N, int nsm) {
-  if (N % 256 != 0) return 128;
-  const long long pairs = static_cast<long long>((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * (N / 256);
+  const long long pairs = static_cast<long long>((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * ((N + 255) / 256);
   if (pairs >= nsm / 2) return BN_PAIR;
+  if (N % 256 != 0) return 128;
   const long long tiles256 = static_cast<long long>((M + GEMM_BM - 1) / GEMM_BM) * (N / 256);
   return tiles256 >= nsm ? 256 : 128;
 }
 
-// Residual GEMMs (proj, FC2): N = D; the paired tile when it fills the SMs, else bn_res (whose
-// half-width fixes the statistics groups, 128 columns for both 256-wide choices).
+// Residual GEMMs (proj, FC2): N = D; the paired tile when D is a multiple of 256 and the pairs
+// fill the SMs, else bn_res (whose half-width fixes the statistics groups).  A padded paired
+// tile was measured slower here than 128 x 128 (ViT-S/16@336 b64 proj 46 against 38 us): the
+// residual epilogue, not the MMA, sets these tiles' pace.
 int pick_bn_res(int M, int D, int bn_res, int nsm) {
   if (bn_res != 256) return bn_res;
   const long long pairs = static_cast<long long>((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * (D / 256);
@@ -639,6 +643,7 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
       ep.x = S.x;
       ep.xb = S.xb;
       ep.stats_out = S.stats;
+      ep.stats_cols = m->stats_cols;
       const int bnr = pick_bn_res(M, D, m->bn_res, m->nsm);
       { const int ps_ = prof_open(m, VIT_K_PROJ_GEMM, s);
       CK(launch_gemm(bnr, EPI_RESID, tm_attn, bnr == BN_PAIR ? bw.tm_proj_h : bw.tm_proj, tm_x_ep, tm_xb_ep, M, D, D, ep,
@@ -677,6 +682,7 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
       ep.x = S.x;
       ep.xb = S.xb;
       ep.stats_out = S.stats;
+      ep.stats_cols = m->stats_cols;
       const int bnr = pick_bn_res(M, D, m->bn_res, m->nsm);
       { const int ps_ = prof_open(m, VIT_K_FC2_GEMM, s);
       CK(launch_gemm(bnr, EPI_RESID, tm_h, bnr == BN_PAIR ? bw.tm_fc2_h : bw.tm_fc2, tm_x_ep, tm_xb_ep, M, D, F, ep,
