@@ -84,6 +84,30 @@ __device__ __forceinline__ void merge_stats(float& n, float& mean, float& m2, fl
   n = tot;
 }
 
+// Mean and sum of squared deviations of 32 values, in four interleaved chains (the sum first,
+// then the deviations from the mean): short dependency chains for the residual epilogue.
+__device__ __forceinline__ void chunk_mean_m2(const float (&v)[32], float& mean, float& m2) {
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    s0 += v[j];
+    s1 += v[j + 1];
+    s2 += v[j + 2];
+    s3 += v[j + 3];
+  }
+  mean = ((s0 + s1) + (s2 + s3)) * (1.0f / 32.0f);
+  float q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    const float d0 = v[j] - mean, d1 = v[j + 1] - mean, d2 = v[j + 2] - mean, d3 = v[j + 3] - mean;
+    q0 = fmaf(d0, d0, q0);
+    q1 = fmaf(d1, d1, q1);
+    q2 = fmaf(d2, d2, q2);
+    q3 = fmaf(d3, d3, q3);
+  }
+  m2 = (q0 + q1) + (q2 + q3);
+}
+
 // Affine epilogue of one 32-column chunk for BIAS / LNFOLD: v <- act(rstd * v - rstd * mu * c + b),
 // two columns per packed f32x2 instruction.
 template <int MODE>
@@ -242,18 +266,29 @@ __device__ __forceinline__ void epilogue_resid(const EpiParams& ep, const CUtens
     uint8_t* xr = xbuf0 + buf * 4096 + lane * 128;
     const float4* b4 = reinterpret_cast<const float4*>(ep.bias + n);
     const float4* l4 = reinterpret_cast<const float4*>(ep.ls + n);
+    // every load of the chunk is issued before the first use, so their latencies overlap
+    float4 xo[8], bb[8], ll[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      float4* xp = reinterpret_cast<float4*>(xr + ((k ^ (lane & 7)) << 4));
-      const float4 xo = *xp;
-      const float4 bb = __ldg(b4 + k);
-      const float4 ll = __ldg(l4 + k);
-      v[4 * k + 0] = fmaf(ll.x, v[4 * k + 0] + bb.x, xo.x);
-      v[4 * k + 1] = fmaf(ll.y, v[4 * k + 1] + bb.y, xo.y);
-      v[4 * k + 2] = fmaf(ll.z, v[4 * k + 2] + bb.z, xo.z);
-      v[4 * k + 3] = fmaf(ll.w, v[4 * k + 3] + bb.w, xo.w);
-      *xp = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+      xo[k] = *reinterpret_cast<const float4*>(xr + ((k ^ (lane & 7)) << 4));
+      bb[k] = __ldg(b4 + k);
+      ll[k] = __ldg(l4 + k);
     }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float2 a0 = fadd2(make_float2(v[4 * k + 0], v[4 * k + 1]), make_float2(bb[k].x, bb[k].y));
+      const float2 a1 = fadd2(make_float2(v[4 * k + 2], v[4 * k + 3]), make_float2(bb[k].z, bb[k].w));
+      const float2 r0 = ffma2(make_float2(ll[k].x, ll[k].y), a0, make_float2(xo[k].x, xo[k].y));
+      const float2 r1 = ffma2(make_float2(ll[k].z, ll[k].w), a1, make_float2(xo[k].z, xo[k].w));
+      v[4 * k + 0] = r0.x;
+      v[4 * k + 1] = r0.y;
+      v[4 * k + 2] = r1.x;
+      v[4 * k + 3] = r1.y;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      *reinterpret_cast<float4*>(xr + ((k ^ (lane & 7)) << 4)) =
+          make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       uint4 w;
@@ -270,16 +305,8 @@ __device__ __forceinline__ void epilogue_resid(const EpiParams& ep, const CUtens
       tma_store_2d(tmXb, xbbuf, n, row0);
       tma_store_commit();
     }
-    float s = 0.f;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) s += v[j];
-    const float cm = s * (1.0f / 32.0f);
-    float q = 0.f;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float d = v[j] - cm;
-      q = fmaf(d, d, q);
-    }
+    float cm, q;
+    chunk_mean_m2(v, cm, q);
     merge_stats(run_n, run_mean, run_m2, 32.f, cm, q);
     if ((n + 32) % ep.stats_cols == 0) {
       if (row < ep.M)
