@@ -173,3 +173,40 @@ def test_nonfinite_input_is_reported_by_poll():
     enc.forward(im)
     enc.poll()                                  # flag cleared
     enc.close()
+
+
+def test_forward_rejects_bad_arguments():
+    """vit_forward validates on the host before any launch: a batch outside 1..max_batch, a
+    workspace below vit_workspace_size and pointers that are not 16-byte aligned are refused with
+    their status codes, and the model still gives the same descriptors afterwards."""
+    need_cuda()
+    import ctypes
+    import vision_transformer_encoder_fwd_b200 as V
+    spec = S.PRESETS["tiny_s16"]
+    enc = V.VitEncoder(spec, S.make_weights(spec, 61), max_batch=2)
+    im = S.make_images(spec, 3, 62).cuda().contiguous()
+    before = enc.forward(im[:2], desc=True)["desc"].clone()
+    desc = torch.empty(2, spec.dim, dtype=torch.float32, device="cuda")
+    need = enc.workspace_size(2)
+    ws = torch.empty(need + 256, dtype=torch.uint8, device="cuda")
+
+    def call(img_ptr, B, ws_bytes, desc_ptr):
+        o = V.VitOutputs()
+        o.desc = desc_ptr
+        return enc.lib.vit_forward(enc.handle, ctypes.c_void_p(img_ptr), B, ctypes.byref(o),
+                                   ctypes.c_void_p(ws.data_ptr()), ws_bytes, None)
+
+    ok_img, ok_desc = im.data_ptr(), desc.data_ptr()
+    assert call(ok_img, 0, need, ok_desc) == V.VIT_E_SHAPE
+    assert call(ok_img, 3, need, ok_desc) == V.VIT_E_SHAPE
+    assert call(ok_img, 2, need - 1, ok_desc) == V.VIT_E_WORKSPACE
+    assert call(ok_img + 4, 2, need, ok_desc) == V.VIT_E_INVALID_ARG
+    assert call(ok_img, 2, need, ok_desc + 4) == V.VIT_E_INVALID_ARG
+    assert call(0, 2, need, ok_desc) == V.VIT_E_INVALID_ARG
+    torch.cuda.synchronize()
+    enc.poll()
+    assert call(ok_img, 2, need, ok_desc) == V.VIT_OK
+    torch.cuda.synchronize()
+    enc.poll()
+    assert torch.equal(desc, before)
+    enc.close()
