@@ -494,7 +494,9 @@ def report(args, spec, wl, B, world, prof, ms_total, value, e2e, launches_per_st
                    "timing": "CUDA events on the launching stream; per-launch events recorded inside the "
                              "timed region for the kernel breakdown"},
         "tflops_per_gpu": step_flops / (ms_total / args.steps / 1000.0) / 1e12,
-        "frac_of_bf16_peak": {"measured_burst": step_flops / (ms_total / args.steps / 1000.0) / 1e12 /
+        "frac_of_bf16_peak": {"measured_sustained": step_flops / (ms_total / args.steps / 1000.0) / 1e12 /
+                              peaks["bf16_tflops_sustained"],
+                              "measured_burst": step_flops / (ms_total / args.steps / 1000.0) / 1e12 /
                               peaks["bf16_tflops"], "spec_dense_2250": step_flops / (
                                   ms_total / args.steps / 1000.0) / 1e12 / 2250.0},
         "roofline": roof,
