@@ -380,6 +380,32 @@ def test_slide_constant_cos_gives_uniform_probs():
     assert np.abs(probs - 1.0 / C).max() < 1e-15 and (lab == 0).all()
 
 
+@pytest.mark.parametrize("H,W", [(80, 144), (80, 150)])
+def test_slide_crops_are_the_windows_in_row_major_order(H, W):
+    """seg_slide's crop loop against crops cut independently: torch's unfold over rows, then over
+    columns, for the regular part of the grid, and explicit slicing from the right edge for the
+    last, clamped column of windows.  A non-square image, so a swapped y / x or a wrong window
+    order changes which pixels a window sees."""
+    spec = S.PRESETS["tiny_s16"]
+    side, stride = 48, 32
+    w = O.to_f64_weights(S.make_weights(spec, 131))
+    img = S.make_images(spec, 1, 132, H, W)[0]
+    text = S.make_text_feats(3, spec.dim, 133)
+    _, _, toks = O.seg_slide(img, w, spec, text, side, stride)
+    ys, xs = O.window_origins(H, side, stride), O.window_origins(W, side, stride)
+    assert toks.shape[0] == len(ys) * len(xs)
+    grid = img.unfold(1, side, stride).unfold(2, side, stride)      # [3, nY, nX, side, side]
+    for iy, y in enumerate(ys):
+        for ix, x in enumerate(xs):
+            if ix < grid.shape[2] and x == ix * stride:
+                crop = grid[:, iy, ix]
+            else:                                                   # the clamped last column
+                assert x == W - side
+                crop = img[:, y:y + side, W - side:]
+            ref = O.forward(crop[None].contiguous(), w, spec)["patch_tokens"][0]
+            assert np.array_equal(toks[iy * len(xs) + ix], ref), (iy, ix)
+
+
 def test_cos_map_is_cosine():
     rng = np.random.default_rng(21)
     toks = rng.standard_normal((6, 10)) * 5
