@@ -55,3 +55,28 @@ def test_report_line_carries_the_contract_keys():
     assert line["frac_of_bf16_peak"]["measured_sustained"] == pytest.approx(step_tflops / 1397.0)
     assert line["frac_of_bf16_peak"]["spec_dense_2250"] == pytest.approx(step_tflops / 2250.0)
     assert line["kernels"]["final_ln"]["gbs"] > 0
+
+
+def test_cpu_baseline_decomposition_matches_a_full_oracle_run():
+    """The CPU baseline times the oracle's per-image work outside the blocks once (the patch
+    embedding on a strip, scaled by the patch count) plus one block counted depth times; on a
+    small encoder that sum must agree with a full oracle forward to within timing noise."""
+    import time
+    import oracle as O
+    spec = S.PRESETS["small_s16"]
+    w = O.to_f64_weights(S.make_weights(spec, 3))
+    im = S.make_images(spec, 1, 4)
+    best_full = min(_timed(lambda: O.forward(im, w, spec)) for _ in range(3))
+    est = []
+    for _ in range(3):
+        t_fixed, desc = bench.oracle_fixed_part(spec, w, im)
+        est.append(t_fixed + spec.depth * bench.oracle_block_time(spec, w))
+    assert "patch rows" in desc
+    assert 0.33 * best_full <= min(est) <= 3.0 * best_full, (min(est), best_full)
+
+
+def _timed(fn):
+    import time
+    t0 = time.perf_counter()
+    fn()
+    return time.perf_counter() - t0
