@@ -257,8 +257,10 @@ vit_status vit_seg_zero_shot(vit_model *m, const float *image, int32_t H, int32_
  *   and a message naming the size (ViT-S/16 at 336 x 336 needs about 2.8 MB per image, so up
  *   to 24 images fit; ViT-L/16 at 1024 x 1024 needs 67.5 MB and does not fit even one image).
  *   Every GPU that loads the library holds the 64 MiB until the process exits.
- *   The first call on each device looks up the array's device address (cudaGetSymbolAddress)
- *   with that device current; make that first call before any stream capture.
+ *   vit_create looks up the array's device address (cudaGetSymbolAddress) on the model's
+ *   device, with that device current, so a call never does that lookup itself.  The model's
+ *   device must be current when this is called (VIT_E_INVALID_ARG otherwise, before any
+ *   launch), so the array of another GPU is never paired with this model's weights.
  *   All calls share the one array, on every stream and model: calls whose work overlaps on
  *   the GPU race on it and must be serialised by the caller.  Nothing in it needs to start at
  *   zero; each call overwrites what it reads. */
@@ -270,6 +272,15 @@ vit_status vit_forward_noalloc(vit_model *m, const float *images, int32_t B, con
  * VIT_E_NONFINITE if a token row reaching the final LayerNorm held a NaN or an infinity, or
  * VIT_E_CUDA if the stream reports an error. */
 vit_status vit_poll(vit_model *m, vit_stream_t stream);
+
+/* Limit, in nanoseconds, of every pipeline wait in the model's later launches (0 restores the
+ * default of 2 s, far above any real wait).  A wait that runs out makes its kernel record
+ * VIT_E_DEVICE_TIMEOUT for vit_poll, let the copies and MMAs it has in flight land, free its
+ * tensor memory and return; the kernels launched after it on the model find the status word
+ * set and return without work until vit_poll clears it.  A limit shorter than the pipeline's
+ * latency therefore exercises that path on purpose (the failure-detection test does this).
+ * Host-side setting only: no launch, no synchronisation. */
+vit_status vit_set_wait_limit(vit_model *m, uint64_t ns);
 
 /* Number of kernel launches the last vit_forward / vit_forward_hw / vit_seg_zero_shot call made. */
 int32_t vit_last_launch_count(const vit_model *m);

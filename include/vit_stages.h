@@ -23,12 +23,24 @@ extern "C" {
 vit_status vit_stage_linear(const void *A, const void *W, const float *bias, int32_t M, int32_t N, int32_t K,
                             int32_t gelu, void *out, int32_t *status, vit_stream_t stream);
 
+/* vit_stage_linear with the limit of its pipeline waits given in nanoseconds (0: the default 2 s);
+ * vit_stage_linear is this with 0.  When a wait runs out the kernel writes a non-zero code into
+ * *status, lets its copies and MMAs in flight land, frees its tensor memory and returns. */
+vit_status vit_stage_linear_bounded(const void *A, const void *W, const float *bias, int32_t M, int32_t N,
+                                    int32_t K, int32_t gelu, void *out, int32_t *status, uint64_t wait_ns,
+                                    vit_stream_t stream);
+
 /* Multi-head self-attention core ("DINOv2 n semantic" diagram, "Encoder self-attention"):
  * for each image b and head h, out[b, :, 64h:64h+64] = softmax_keys(Q_h K_h^T / 8) V_h with
  * Q_h, K_h, V_h the 64-column slices h of the q, k and v parts of qkv[b] = [q | k | v].
  *   qkv: bf16 [B, T, 3 * 64 * heads];  out: bf16 [B, T, 64 * heads].  T >= 1, heads >= 1. */
 vit_status vit_stage_attention(const void *qkv, int32_t B, int32_t T, int32_t heads, void *out, int32_t *status,
                                vit_stream_t stream);
+
+/* vit_stage_attention with the limit of its pipeline waits given in nanoseconds (0: the default
+ * 2 s), with the same behaviour on expiry as vit_stage_linear_bounded. */
+vit_status vit_stage_attention_bounded(const void *qkv, int32_t B, int32_t T, int32_t heads, void *out,
+                                       int32_t *status, uint64_t wait_ns, vit_stream_t stream);
 
 /* GELU as the FC1 epilogue evaluates it ([diagram] "Encoder block": exact erf form, with erf from
  * Abramowitz & Stegun 7.1.28, absolute error <= 1.5e-7 |x| plus fp32 rounding):

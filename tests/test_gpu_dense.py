@@ -2,9 +2,12 @@
 Bottleneck", "Projector output ConvX", "Task head") through vit_set_dense_head /
 vit_forward_dense, against the fp64 oracle's dense_head on the oracle's own taps.
 
-Tolerance: the GPU keeps the activations between convs in bf16 (fp32 accumulation and
-statistics) across ten conv / norm stages, so projector features and logits are compared at
-3e-2 of their largest magnitude (the per-block bar, widened for the longer bf16 chain)."""
+Tolerance: projector features and logits within 2e-2 of their largest magnitude (the encoder's
+per-block bar), although the GPU keeps the activations between the ten conv / norm stages in
+bf16 (fp32 accumulation and statistics).  Class agreement: the seeded head gives nearly flat
+logits over 19 classes, so many pixels have two classes within the error bar of each other;
+there both answers are right at the stated precision.  The argmax must agree on at least 99.5%
+of the pixels whose top-2 gap exceeds twice the error bar, and on at least 99% of all pixels."""
 import numpy as np
 import pytest
 import torch
@@ -14,7 +17,7 @@ import synthetic as S
 from parity import block_rel_err, gpu, need_cuda
 
 pytestmark = gpu
-DENSE_REL_MAX = 3e-2
+DENSE_REL_MAX = 2e-2
 
 
 def _check(spec, w, hw, im, idx, out_hw):
@@ -34,10 +37,18 @@ def _check(spec, w, hw, im, idx, out_hw):
     for j, i in enumerate(idx):
         ep = block_rel_err(g_p4[i], ref["p4"][j])
         el = block_rel_err(g_logits[i], ref["logits"][j])
+        r = ref["logits"][j]
+        agree = (g_logits[i].argmax(0) == r.argmax(0)).mean()
+        top2 = np.sort(r, axis=0)[-2:]
+        clear = (top2[1] - top2[0]) > 2 * DENSE_REL_MAX * np.abs(r).max()
+        agree_clear = (g_logits[i].argmax(0) == r.argmax(0))[clear].mean()
+        print(f"dense head image {i}: p4 rel err {ep:.3e}, logits rel err {el:.3e}, argmax agreement "
+              f"{agree:.5f} (all pixels), {agree_clear:.5f} on the {clear.mean():.3f} of pixels whose top-2 gap "
+              f"exceeds twice the tolerance")
         assert ep <= DENSE_REL_MAX, f"image {i}: projector rel err {ep:.3e}"
         assert el <= DENSE_REL_MAX, f"image {i}: logits rel err {el:.3e}"
-        agree = (g_logits[i].argmax(0) == ref["logits"][j].argmax(0)).mean()
-        assert agree >= 0.98, agree
+        assert agree_clear >= 0.995, agree_clear
+        assert agree >= 0.99, agree
     return n_launch
 
 

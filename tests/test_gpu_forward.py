@@ -66,6 +66,67 @@ def test_vitl16_1024_b8():
     assert_forward_parity(g, ref, spec, idx)
 
 
+@pytest.mark.slow
+def test_vitl16_1024_b1():
+    """ViT-L/16@1024, batch 1: the batch of the DINOv3 deployment article's latency table (§3.2).
+    At M = 4,101 rows the residual GEMMs run on single-CTA 128 x 256 tiles, not the paired tiles
+    that batch 8 takes, so this shape is checked on its own."""
+    need_cuda()
+    spec, w, im = S.make_workload("vitl16_1024_b1")
+    g = run_gpu(spec, w, im, hidden=True)
+    assert np.isfinite(g["hidden"]).all()
+    ref = O.forward(im, w, spec, record_hidden=True)
+    assert_forward_parity(g, ref, spec, [0])
+
+
+def _ln_rows(x):
+    """Plain per-row LayerNorm (no affine), fp64: what a folded LayerNorm hands its GEMM."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(-1, keepdims=True)
+    return (x - mu) / np.sqrt(((x - mu) ** 2).mean(-1, keepdims=True) + 1e-6)
+
+
+def _offset_rows(spec, w, seed):
+    """CLS and register rows (and, through the patch bias, every patch row) whose mean is large
+    against their spread.  kornia/dinov3 card, "Build BF16, not FP16": activations of the encoder
+    stay below ~1.8e3, so the largest offset here is 1,500."""
+    g = torch.Generator().manual_seed(seed)
+    D = spec.dim
+    w = dict(w)
+    w["cls"] = S.to_bf16(15.0 + 1.5 * torch.randn(D, generator=g))
+    if spec.registers:
+        offs = [150.0, 1500.0, -150.0] + [0.0] * (spec.registers - 3)
+        reg = torch.stack([o + 1.5 * torch.randn(D, generator=g) for o in offs[:spec.registers]])
+        w["reg"] = S.to_bf16(reg)
+    w["patch_b"] = S.to_bf16(w["patch_b"].float() + 20.0)
+    return w
+
+
+@pytest.mark.parametrize("name", ["tiny_s16", "small_s16", "vitb14_224"])
+def test_rows_with_large_mean(name):
+    """The folded LayerNorm multiplies a bf16 copy of the residual stream.  Rows whose mean is
+    large against their spread (|mean|/std from ~10 to several hundred here) lose their spread
+    to bf16 rounding unless that copy is re-centred; the check is on what the LayerNorm sees:
+    every row of every block's output, normalised, against the oracle's."""
+    need_cuda()
+    spec = S.PRESETS[name]
+    w = _offset_rows(spec, S.make_weights(spec, 83), 84)
+    im = S.make_images(spec, 2, 85)
+    g = run_gpu(spec, w, im)
+    ref = O.forward(im, w, spec, record_hidden=True)
+    assert_forward_parity(g, ref, spec, [0, 1])
+    ratio = 0.0
+    for l in range(spec.depth):
+        for i in range(2):
+            xr = ref["hidden"][l, i]
+            r = np.abs(xr.mean(-1)) / xr.std(-1)
+            ratio = max(ratio, float(r.max()))
+            a, b = _ln_rows(g["hidden"][l, i]), _ln_rows(xr)
+            err = np.abs(a - b).max(-1) / np.abs(b).max(-1)
+            assert err.max() <= 2e-2, f"block {l + 1} image {i}: row {int(err.argmax())} normalised rel err {err.max():.3e}"
+    assert ratio >= (300.0 if spec.registers else 5.0), ratio
+
+
 def test_forward_host_matches_device_path():
     need_cuda()
     import vision_transformer_encoder_fwd_b200 as V

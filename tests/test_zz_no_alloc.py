@@ -50,17 +50,53 @@ def test_noalloc_matches_vit_forward_twice():
     enc.close()
 
 
-def test_noalloc_refuses_batches_beyond_the_fixed_scratch():
+NOALLOC_BYTES = 64 << 20        # the fixed array's size, as the header states
+NOALLOC_VITS16_336_MAX_BATCH = 24  # the largest ViT-S/16@336 batch the header says fits
+
+
+def test_noalloc_boundary_of_the_fixed_scratch():
+    """The largest batch whose workspace fits the fixed array runs and matches vit_forward; one
+    image more is refused with VIT_E_WORKSPACE before anything is launched."""
     need_cuda()
     import vision_transformer_encoder_fwd_b200 as V
     spec = S.VITS16_336
-    B = 32                     # about 88 MB of workspace, above the fixed 64 MiB
-    enc = V.VitEncoder(spec, S.make_weights(spec, 93), max_batch=B)
-    assert enc.workspace_size(B) > (64 << 20)
-    images = torch.zeros(B, 3, spec.img_h, spec.img_w, device="cuda")
-    outs = enc.alloc_outputs(B, desc=True, patch=True, patch_fp32=True)
+    enc = V.VitEncoder(spec, S.make_weights(spec, 93), max_batch=40)
+    bmax = max(b for b in range(1, 41) if enc.workspace_size(b) <= NOALLOC_BYTES)
+    assert bmax == NOALLOC_VITS16_336_MAX_BATCH, bmax
     lib = V.load_library()
-    st = lib.vit_forward_noalloc(enc.handle, images.data_ptr(), B, ctypes.byref(_outputs(V, outs)), None)
+    big = torch.zeros(bmax + 1, 3, spec.img_h, spec.img_w, device="cuda")
+    outs = enc.alloc_outputs(bmax + 1, desc=True, patch=True, patch_fp32=True)
+    st = lib.vit_forward_noalloc(enc.handle, big.data_ptr(), bmax + 1, ctypes.byref(_outputs(V, outs)), None)
     assert st == V.VIT_E_WORKSPACE
     assert b"fixed" in lib.vit_last_error()
+    images = S.make_images(spec, bmax, 94).cuda()
+    ref = enc.forward(images, desc=True, patch=True, patch_fp32=True)
+    got = enc.alloc_outputs(bmax, desc=True, patch=True, patch_fp32=True)
+    st = lib.vit_forward_noalloc(enc.handle, images.data_ptr(), bmax, ctypes.byref(_outputs(V, got)), None)
+    assert st == V.VIT_OK, lib.vit_last_error()
+    torch.cuda.synchronize()
+    enc.poll()
+    assert torch.equal(got["desc"], ref["desc"])
+    assert torch.equal(got["patch_tokens"], ref["patch_tokens"])
+    enc.close()
+
+
+def test_noalloc_refuses_another_current_device():
+    """With another GPU current the call is refused before any launch: the fixed array of that GPU
+    must never be paired with this model's weights."""
+    need_cuda()
+    if torch.cuda.device_count() < 2:
+        import pytest
+        pytest.skip("needs two visible GPUs")
+    import vision_transformer_encoder_fwd_b200 as V
+    spec = S.PRESETS["tiny_s16"]
+    torch.cuda.set_device(0)
+    enc = V.VitEncoder(spec, S.make_weights(spec, 95), max_batch=1)
+    images = S.make_images(spec, 1, 96).cuda(0)
+    outs = enc.alloc_outputs(1, desc=True, patch=True, patch_fp32=True)
+    lib = V.load_library()
+    with torch.cuda.device(1):
+        st = lib.vit_forward_noalloc(enc.handle, images.data_ptr(), 1, ctypes.byref(_outputs(V, outs)), None)
+    assert st == V.VIT_E_INVALID_ARG
+    assert b"device" in lib.vit_last_error()
     enc.close()

@@ -97,7 +97,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "vit_profile_begin": (I32, [P, I32]),
         "vit_profile_end": (I32, [P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(I32)]),
         "vit_stage_linear": (I32, [P, P, P, I32, I32, I32, I32, P, P, P]),
+        "vit_stage_linear_bounded": (I32, [P, P, P, I32, I32, I32, I32, P, P, ctypes.c_uint64, P]),
         "vit_stage_attention": (I32, [P, I32, I32, I32, P, P, P]),
+        "vit_stage_attention_bounded": (I32, [P, I32, I32, I32, P, P, ctypes.c_uint64, P]),
+        "vit_set_wait_limit": (I32, [P, ctypes.c_uint64]),
         "vit_stage_pos_resize": (I32, [P, I32, I32, I32, I32, I32, I32, P, P]),
         "vit_stage_gelu": (I32, [P, ctypes.c_int64, P, P]),
     }
@@ -347,6 +350,10 @@ class VitEncoder:
             wsb.numel(), _stream_handle(stream)))
         return p, lb
 
+    def set_wait_limit(self, ns: int) -> None:
+        """vit_set_wait_limit: the limit of every pipeline wait of later launches (0: 2 s)."""
+        _check("vit_set_wait_limit", self.lib.vit_set_wait_limit(self.handle, int(ns)))
+
     def poll(self, stream=None) -> None:
         _check("vit_poll", self.lib.vit_poll(self.handle, _stream_handle(stream)))
 
@@ -377,8 +384,9 @@ class VitEncoder:
 
 
 # ------------------------------------------------------------------ stage entry points
-def stage_linear(A, W, bias, gelu: bool = False, out=None, status=None, stream=None):
-    """vit_stage_linear: out = act(A W^T + bias), bf16 in/out, fp32 bias."""
+def stage_linear(A, W, bias, gelu: bool = False, out=None, status=None, stream=None, wait_ns: int = 0):
+    """vit_stage_linear(_bounded): out = act(A W^T + bias), bf16 in/out, fp32 bias; wait_ns > 0
+    sets the limit of the kernel's pipeline waits."""
     import torch
     lib = load_library()
     M, K = A.shape
@@ -386,21 +394,22 @@ def stage_linear(A, W, bias, gelu: bool = False, out=None, status=None, stream=N
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=A.device)
     st = status if status is not None else torch.zeros(1, dtype=torch.int32, device=A.device)
-    _check("vit_stage_linear", lib.vit_stage_linear(_ptr(A), _ptr(W), _ptr(bias), M, N, K, 1 if gelu else 0,
-                                                    _ptr(out), _ptr(st), _stream_handle(stream)))
+    _check("vit_stage_linear", lib.vit_stage_linear_bounded(_ptr(A), _ptr(W), _ptr(bias), M, N, K, 1 if gelu else 0,
+                                                            _ptr(out), _ptr(st), int(wait_ns), _stream_handle(stream)))
     return out, st
 
 
-def stage_attention(qkv, heads: int, out=None, status=None, stream=None):
-    """vit_stage_attention: qkv bf16 [B, T, 3 * 64 * heads] -> out bf16 [B, T, 64 * heads]."""
+def stage_attention(qkv, heads: int, out=None, status=None, stream=None, wait_ns: int = 0):
+    """vit_stage_attention(_bounded): qkv bf16 [B, T, 3 * 64 * heads] -> out bf16 [B, T, 64 * heads];
+    wait_ns > 0 sets the limit of the kernel's pipeline waits."""
     import torch
     lib = load_library()
     B, T, _ = qkv.shape
     if out is None:
         out = torch.empty(B, T, heads * 64, dtype=torch.bfloat16, device=qkv.device)
     st = status if status is not None else torch.zeros(1, dtype=torch.int32, device=qkv.device)
-    _check("vit_stage_attention", lib.vit_stage_attention(_ptr(qkv), B, T, heads, _ptr(out), _ptr(st),
-                                                          _stream_handle(stream)))
+    _check("vit_stage_attention", lib.vit_stage_attention_bounded(_ptr(qkv), B, T, heads, _ptr(out), _ptr(st),
+                                                                  int(wait_ns), _stream_handle(stream)))
     return out, st
 
 

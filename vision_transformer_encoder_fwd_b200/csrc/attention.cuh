@@ -141,7 +141,8 @@ __device__ __forceinline__ void softmax_block_p(const float (&s)[128], float mc,
 
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __nv_bfloat16* __restrict__ qkv, int T, int D,
-                       __nv_bfloat16* __restrict__ out, int* gstatus) {
+                       __nv_bfloat16* __restrict__ out, int* gstatus, unsigned long long wait_ns) {
+  const unsigned long long wlim = wait_limit(wait_ns);
   extern __shared__ __align__(1024) uint8_t smem[];
   // The swizzled layouts assume 1024-byte aligned tiles; report and stop if the shared window
   // is not (uniform across the CTA, before anything is allocated).
@@ -215,7 +216,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     for (int j = 0; j < nkv; ++j) {
       const int s = j % ATT_KV_STAGES;
       const uint32_t ph = static_cast<uint32_t>(j / ATT_KV_STAGES) & 1u;
-      if (!mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 1)) break;
+      if (!mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 1, wlim)) break;
       mbar_arrive_expect_tx(&kv_full[s], AttnCfg::K_BYTES + AttnCfg::V_BYTES);
       tma_load_3d(sK + s * AttnCfg::K_BYTES, &tmQKV, D + h * 64, j * ATT_BN, b, &kv_full[s]);
       tma_load_3d(sV + s * AttnCfg::V_BYTES, &tmQKV, 2 * D + h * 64, j * ATT_BN, b, &kv_full[s]);
@@ -260,8 +261,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) ap[i][kk] = t_s0 + i * 128 + kk * 8;
       }
-      bool ok = mbar_wait(q_ready, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 2) &&
-                mbar_wait(&kv_full[0], 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 3);
+      bool ok = mbar_wait(q_ready, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 2, wlim) &&
+                mbar_wait(&kv_full[0], 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 3, wlim);
       if (ok) {
         tc_fence_after();
         for (int i = 0; i < ntile; ++i) {
@@ -280,7 +281,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         for (int i = 0; i < ntile && ok; ++i) {
           // P arrives in two halves of 64 keys: the first four PV MMAs run while the softmax
           // group is still producing the second half.
-          if (!mbar_wait(&p_full[2 * i], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 4)) {
+          if (!mbar_wait(&p_full[2 * i], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 4, wlim)) {
             ok = false;
             break;
           }
@@ -290,7 +291,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             const uint64_t b_lo[4] = {dvs[0], dvs[1], dvs[2], dvs[3]};
             tc_mma_ts_chain4(t_o0 + i * AttnCfg::O_COLS, a_lo, b_lo, idesc_o, j > 0 ? 1u : 0u);
           }
-          if (!mbar_wait(&p_full[2 * i + 1], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 9)) {
+          if (!mbar_wait(&p_full[2 * i + 1], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 9, wlim)) {
             ok = false;
             break;
           }
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           if (j + 1 < nkv) {
             if (i == 0) {
               if (!mbar_wait(&kv_full[s1], static_cast<uint32_t>((j + 1) / ATT_KV_STAGES) & 1u, abort_flag, gstatus,
-                             DEV_TIMEOUT_ATTN + 5)) {
+                             DEV_TIMEOUT_ATTN + 5, wlim)) {
                 ok = false;
                 break;
               }
@@ -354,7 +355,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       float m = -INFINITY;
       bool ok = true;
       for (int j = 0; j < nkv; ++j) {
-        if (!mbar_wait(&s_full[wg], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 6)) {
+        if (!mbar_wait(&s_full[wg], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 6, wlim)) {
           ok = false;
           break;
         }
@@ -379,7 +380,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           // O_i holds the blocks before j at the old maximum: wait for the last of them, rescale
           // (the sum column included) before any P of block j is released to the MMA.
           if (!mbar_wait(&pv_done[wg], static_cast<uint32_t>(j - 1) & 1u, abort_flag, gstatus,
-                         DEV_TIMEOUT_ATTN + 7)) {
+                         DEV_TIMEOUT_ATTN + 7, wlim)) {
             ok = false;
             break;
           }
@@ -402,7 +403,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         else
           softmax_block_p<false>(s, mc, valid, t_s, &p_full[2 * wg], &p_full[2 * wg + 1]);
       }
-      if (ok && mbar_wait(mma_done, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 8)) {
+      if (ok && mbar_wait(mma_done, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 8, wlim)) {
         tc_fence_after();
         float o[64], lsum[16];
         __syncwarp();

@@ -66,32 +66,64 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// CLS and register rows of the residual stream ([card] "Model I/O": CLS, then 4 registers;
-// [diagram] position embedding row 0 on CLS for DINOv2): x, its bf16 copy and the per-group
-// (mean, M2) statistics the folded LayerNorm of block 1 reads.  grid (ngroups, 1 + R, B),
-// one warp per (row, column group of gcols).
-__global__ void prefix_tokens_kernel(const float* __restrict__ cls, const float* __restrict__ reg,
-                                     const float* __restrict__ pos, int pos_on_cls, int T, int D, int gcols,
-                                     float* __restrict__ x, __nv_bfloat16* __restrict__ xb, float2* __restrict__ stats) {
-  const int g = blockIdx.x, t = blockIdx.y, b = blockIdx.z;
-  const int lane = threadIdx.x;
-  const size_t row = static_cast<size_t>(b) * T + t;
-  float s = 0.f;
-  for (int j = lane; j < gcols; j += 32) {
-    const int n = g * gcols + j;
-    float v = (t == 0) ? cls[n] + (pos_on_cls ? pos[n] : 0.f) : reg[static_cast<size_t>(t - 1) * D + n];
-    x[row * D + n] = v;
-    xb[row * D + n] = __float2bfloat16_rn(v);
-    s += v;
+// Token rows of the residual stream before block 1, whole rows at a time: the CLS and register
+// rows are written here ([card] "Model I/O": CLS, then the registers, no position embedding on
+// them; [diagram] position embedding row 0 on CLS for DINOv2), the patch rows were written by
+// the patch GEMM.  For every row this kernel then writes what the folded LayerNorm of block 1
+// reads: the (mean, M2) partial statistics of each group of gcols columns, the row mean as the
+// centre, and the re-centred bf16 copy xb = bf16(x - centre).  One warp per row; lane l owns
+// the columns 128 c + 4 l .. + 3 (float4 accesses); gcols is 64 or 128.
+__global__ void token_prep_kernel(const float* __restrict__ cls, const float* __restrict__ reg,
+                                  const float* __restrict__ pos, int pos_on_cls, long long rows, int T, int R, int D,
+                                  int gcols, float* __restrict__ x, __nv_bfloat16* __restrict__ xb,
+                                  float2* __restrict__ stats, float* __restrict__ ctr) {
+  const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int lane = threadIdx.x & 31;
+  const int t = static_cast<int>(row % T);
+  float* xr = x + static_cast<size_t>(row) * D;
+  const int lpg = gcols / 4;  // lanes per statistics group within a 128-column chunk
+  const int ng = D / gcols;
+  float lsum = 0.f;
+  for (int c = 0; c < D / 128; ++c) {
+    const int n = c * 128 + lane * 4;
+    float4 v;
+    if (t <= R) {
+      if (t == 0) {
+        v = *reinterpret_cast<const float4*>(cls + n);
+        if (pos_on_cls) {
+          const float4 p = *reinterpret_cast<const float4*>(pos + n);
+          v.x += p.x;
+          v.y += p.y;
+          v.z += p.z;
+          v.w += p.w;
+        }
+      } else {
+        v = *reinterpret_cast<const float4*>(reg + static_cast<size_t>(t - 1) * D + n);
+      }
+      *reinterpret_cast<float4*>(xr + n) = v;
+    } else {
+      v = *reinterpret_cast<const float4*>(xr + n);
+    }
+    float s = (v.x + v.y) + (v.z + v.w);
+    lsum += s;
+    for (int o = lpg / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float gm = s / static_cast<float>(gcols);
+    const float d0 = v.x - gm, d1 = v.y - gm, d2 = v.z - gm, d3 = v.w - gm;
+    float q = (d0 * d0 + d1 * d1) + (d2 * d2 + d3 * d3);
+    for (int o = lpg / 2; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    if (lane % lpg == 0) stats[static_cast<size_t>(row) * ng + (n / gcols)] = make_float2(gm, q);
   }
-  const float mean = warp_sum(s) / static_cast<float>(gcols);
-  float q = 0.f;
-  for (int j = lane; j < gcols; j += 32) {
-    const float d = x[row * D + g * gcols + j] - mean;
-    q = fmaf(d, d, q);
+  const float centre = warp_sum(lsum) / static_cast<float>(D);
+  for (int c = 0; c < D / 128; ++c) {
+    const int n = c * 128 + lane * 4;
+    const float4 v = *reinterpret_cast<const float4*>(xr + n);
+    uint2 w;
+    w.x = pack_bf16x2(v.x - centre, v.y - centre);
+    w.y = pack_bf16x2(v.z - centre, v.w - centre);
+    *reinterpret_cast<uint2*>(xb + static_cast<size_t>(row) * D + n) = w;
   }
-  q = warp_sum(q);
-  if (lane == 0) stats[row * (D / gcols) + g] = make_float2(mean, q);
+  if (lane == 0) ctr[row] = centre;
 }
 
 // [diagram] "DINOv2-S encoder": the learned position grid goes through "Bicubic
@@ -215,7 +247,7 @@ __global__ void final_ln_kernel(const float* __restrict__ x, const float* __rest
 __global__ void final_ln_stream_kernel(float* __restrict__ x, const float* __restrict__ g,
                                        const float* __restrict__ be, long long rows, int D, float eps, int gcols,
                                        __nv_bfloat16* __restrict__ xb, float2* __restrict__ stats,
-                                       int* __restrict__ nonfinite) {
+                                       float* __restrict__ ctr, int* __restrict__ nonfinite) {
   const int warps_per_block = blockDim.x >> 5;
   const long long row = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -227,6 +259,7 @@ __global__ void final_ln_stream_kernel(float* __restrict__ x, const float* __res
   __syncwarp();
   const int per = gcols / 32;  // 2 or 4
   const int ng = D / gcols;
+  float tot = 0.f;
   for (int gi = 0; gi < ng; ++gi) {
     float v[4];
     float s = 0.f;
@@ -238,7 +271,9 @@ __global__ void final_ln_stream_kernel(float* __restrict__ x, const float* __res
         s += v[j];
       }
     }
-    const float gm = warp_sum(s) / static_cast<float>(gcols);
+    const float gs = warp_sum(s);
+    tot += gs;
+    const float gm = gs / static_cast<float>(gcols);
     float q = 0.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -247,12 +282,16 @@ __global__ void final_ln_stream_kernel(float* __restrict__ x, const float* __res
         const float d = v[j] - gm;
         q = fmaf(d, d, q);
         xr[n] = v[j];
-        xb[static_cast<size_t>(row) * D + n] = __float2bfloat16_rn(v[j]);
       }
     }
     q = warp_sum(q);
     if (lane == 0) stats[static_cast<size_t>(row) * ng + gi] = make_float2(gm, q);
   }
+  // the head's first folded LayerNorm reads the re-centred copy bf16(x - centre), centre = the
+  // normalised row's mean (each lane re-reads the columns it has just written)
+  const float centre = tot / static_cast<float>(D);
+  for (int n = lane; n < D; n += 32) xb[static_cast<size_t>(row) * D + n] = __float2bfloat16_rn(xr[n] - centre);
+  if (lane == 0) ctr[row] = centre;
 }
 
 // The patch rows of the residual stream, fp32: tok[b, p, :] = x[b, 1 + R + p, :] (the dino.txt
@@ -372,71 +411,55 @@ __global__ void bf16_to_f32_kernel(const __nv_bfloat16* __restrict__ src, long l
 }
 
 // ------------------------------------------------------------------ zero-shot scoring
-// dino.txt article, patch/text alignment: F.normalize of each patch token, then
-// einsum("cd,hwd->chw") with the text features.  Step 1: inv_norm[i] = 1 / max(||t_i||, 1e-12),
-// one warp per token.
-__global__ void token_inv_norm_kernel(const float* __restrict__ tok, long long rows, int D, float* __restrict__ inv) {
+// [dinotxt] patch/text alignment: cos[w, c, i] = text[c] . t_i / max(||t_i||, 1e-12) (F.normalize
+// of the patch tokens, then einsum("cd,hwd->chw") with the unit text features), computed on the
+// tensor cores as one bf16 GEMM whose operands carry fp32-grade values: each fp32 value v is split
+// as v = hi + lo with hi = bf16(v) and lo = bf16(v - hi), and the K dimension is tripled so that
+//   [hi_t | hi_t | lo_t] . [hi_c | lo_c | hi_c] = hi_t hi_c + hi_t lo_c + lo_t hi_c,
+// which leaves out only lo_t lo_c (relative 2^-16 of each product) and the bf16 rounding of lo
+// (2^-17): the cosines keep about 16 significant bits instead of bf16's 8.
+//
+// Step 1: the token rows, normalised and split: A3[r] = [hi | hi | lo] of t_r / max(||t_r||, 1e-12)
+// (one warp per row, fp32).
+__global__ void cos_split_tokens_kernel(const float* __restrict__ tok, long long rows, int D,
+                                        __nv_bfloat16* __restrict__ a3) {
   const long long r = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= rows) return;
   const int lane = threadIdx.x & 31;
+  const float* t = tok + r * D;
   float q = 0.f;
+  for (int n = lane; n < D; n += 32) q = fmaf(t[n], t[n], q);
+  const float inv = 1.0f / fmaxf(sqrtf(warp_sum(q)), 1e-12f);
+  __nv_bfloat16* o = a3 + r * 3 * D;
   for (int n = lane; n < D; n += 32) {
-    const float v = tok[r * D + n];
-    q = fmaf(v, v, q);
+    const float v = t[n] * inv;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+    o[n] = hi;
+    o[D + n] = hi;
+    o[2 * D + n] = lo;
   }
-  q = warp_sum(q);
-  if (lane == 0) inv[r] = 1.0f / fmaxf(sqrtf(q), 1e-12f);
 }
 
-// Step 2: cos[w, c, i] = inv[w, i] * sum_d text[c, d] tok[w, i, d], an fp32 SIMT GEMM tile of
-// 64 tokens x 64 classes per block (16 x 16 threads, 4 x 4 outputs each, K staged by 16).
-// fp32 keeps the class ranking exact enough for the argmax (scores differ by ~1e-2).
-__global__ void cos_gemm_kernel(const float* __restrict__ tok, const float* __restrict__ inv,
-                                const float* __restrict__ text, int rows_per_win, long long rows, int C, int D,
-                                float* __restrict__ cosout) {
-  __shared__ float sa[16][64 + 4];
-  __shared__ float sb[16][64 + 4];
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const long long r0 = static_cast<long long>(blockIdx.x) * 64;
-  const int c0 = blockIdx.y * 64;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < D; k0 += 16) {
-    for (int i = threadIdx.x; i < 64 * 16; i += 256) {
-      const int rr = i >> 4, kk = i & 15;
-      const long long r = r0 + rr;
-      sa[kk][rr] = (r < rows) ? tok[r * D + k0 + kk] : 0.f;
-      const int c = c0 + rr;
-      sb[kk][rr] = (c < C) ? text[static_cast<size_t>(c) * D + k0 + kk] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float a[4], bv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = sa[kk][ty * 4 + i];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) bv[i] = sb[kk][tx * 4 + i];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) acc[i][jj] = fmaf(a[i], bv[jj], acc[i][jj]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const long long r = r0 + ty * 4 + i;
-    if (r >= rows) continue;
-    const long long w = r / rows_per_win;
-    const long long pi = r - w * rows_per_win;
-    const float s = inv[r];
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const int c = c0 + tx * 4 + jj;
-      if (c < C) cosout[(w * C + c) * rows_per_win + pi] = acc[i][jj] * s;
-    }
+// Step 2: the class rows, split the other way: B3[c] = [hi | lo | hi] of text[c] for c < C, zero
+// rows up to Cpad (one warp per row).
+__global__ void cos_split_text_kernel(const float* __restrict__ text, int C, int Cpad, int D,
+                                      __nv_bfloat16* __restrict__ b3) {
+  const int c = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (c >= Cpad) return;
+  const int lane = threadIdx.x & 31;
+  __nv_bfloat16* o = b3 + static_cast<size_t>(c) * 3 * D;
+  for (int n = lane; n < D; n += 32) {
+    const float v = (c < C) ? text[static_cast<size_t>(c) * D + n] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+    o[n] = hi;
+    o[D + n] = lo;
+    o[2 * D + n] = hi;
   }
 }
+// Step 3 is the tcgen05 GEMM A3 . B3^T with the EPI_COS epilogue (gemm.cuh), which scatters the
+// fp32 results to cos[w, c, p].
 
 // Bilinear source taps of output index i for an in -> out resize with align_corners=False:
 // src = (i + 0.5) * in / out - 0.5 clamped below at 0; neighbours floor(src) and

@@ -21,6 +21,12 @@ enum DeviceStatus : int {
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s: far above any real wait
 
+// The pipeline-wait limit a launch asked for (0: the default kWaitTimeoutNs).  Waits that drain
+// copies already in flight on the way out of an aborted kernel always use the default.
+__host__ __device__ __forceinline__ unsigned long long wait_limit(unsigned long long ns) {
+  return ns ? ns : kWaitTimeoutNs;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -60,18 +66,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the same phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Limits below this are polled with the non-blocking test and a clock check on every poll
+// (a suspended try_wait could otherwise outlast them).
+constexpr unsigned long long kShortWaitNs = 1000000ull;  // 1 ms
+
 // Wait until the phase of `bar` with parity `parity` has completed.  Gives up (returns false)
-// when the CTA's abort flag is raised by another role or after kWaitTimeoutNs; on its own
-// time-out it raises the abort flag and records `site` in the device status word.
+// when the CTA's abort flag is raised by another role or after `limit_ns`; on its own time-out
+// it raises the abort flag and records `site` in the device status word.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* gstatus, int site) {
+                                          int* gstatus, int site, unsigned long long limit_ns = kWaitTimeoutNs) {
+  if (limit_ns < kShortWaitNs) {
+    const unsigned long long t0 = global_ns();
+    for (;;) {
+      if (mbar_test_wait(bar, parity)) return true;
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        atomicExch(gstatus, site);
+        return false;
+      }
+    }
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0) {
       if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitTimeoutNs) {
+      if (global_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicExch(gstatus, site);
         return false;

@@ -32,9 +32,10 @@ constexpr int GEMM_EPI_THREADS = 32 * GEMM_EPI_WARPS;
 
 enum EpiMode : int {
   EPI_BIAS = 0,    // out_bf16 = act(acc + bias)
-  EPI_LNFOLD = 1,  // out_bf16 = act(rstd * (acc - mean * colsum) + bias)  (LayerNorm folded)
-  EPI_RESID = 2,   // x += ls * (acc + bias); xb = bf16(x); row partial stats of x
-  EPI_PATCH = 3,   // x[token row] = acc + bias + pos; xb; row partial stats
+  EPI_LNFOLD = 1,  // out_bf16 = act(rstd * (acc + (ctr - mean) * colsum) + bias)  (LayerNorm folded)
+  EPI_RESID = 2,   // x += ls * (acc + bias); xb = bf16(x - ctr); ctr; row partial stats of x
+  EPI_PATCH = 3,   // x[token row] = acc + bias + pos (xb, ctr and stats: token_prep_kernel)
+  EPI_COS = 4,     // cos[w, c, p] = acc (fp32, class-major per window; row m = w * P + p, column c)
 };
 
 struct EpiParams {
@@ -42,11 +43,16 @@ struct EpiParams {
   const float* bias;  // [N]
   int gelu;           // BIAS / LNFOLD: apply exact-erf GELU
   int ldo;
-  // LNFOLD: per-row LayerNorm statistics rebuilt from partials written by the producer of x
+  // LNFOLD: per-row LayerNorm statistics rebuilt from partials written by the producer of x.
+  // RESID: stats_in holds the partials of x before the update; their merged mean is the centre
+  // of the new bf16 copy.
   const float* colsum;     // [N] column sums of the gamma-folded weight
   const float2* stats_in;  // [M, nt] (mean, M2) of column groups of nt_cols each (nt_cols = BN/2 of the producer)
   int nt, nt_cols, D;
   float eps;
+  // The bf16 copy of x is stored re-centred, xb = bf16(x - ctr[row]): LNFOLD reads ctr, RESID
+  // writes it (one writer per row: the warps of column group 0).
+  float* ctr;              // [M]
   // RESID / PATCH
   float* x;              // [rows, N] fp32 residual stream (PATCH writes it directly)
   __nv_bfloat16* xb;     // [rows, N] bf16 copy of x (A operand of the next folded GEMM)
@@ -56,6 +62,10 @@ struct EpiParams {
   // PATCH: GEMM row m = b * P + p goes to token row b * T + 1 + R + p, position row p + pos_off
   const float* pos;
   int P, T, R, pos_off;
+  unsigned long long wait_ns;  // pipeline-wait limit (0: the default 2 s)
+  // COS: the cosine map [windows, ncls, P] (P from above); columns >= ncls are padding
+  float* cos;
+  int ncls;
 };
 
 template <int BN, int MODE>
@@ -66,7 +76,8 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   // per epilogue warp: RESID two 32 x 32 fp32 x buffers (128-byte rows, 128B swizzle) and one
   // 32 x 32 bf16 buffer (64-byte rows, 64B swizzle); BIAS / LNFOLD one 32 x 64 bf16 buffer
-  static constexpr int EPI_WARP_BYTES = (MODE == EPI_RESID) ? (2 * 4096 + 2048) : (MODE == EPI_PATCH ? 0 : 4096);
+  static constexpr int EPI_WARP_BYTES =
+      (MODE == EPI_RESID) ? (2 * 4096 + 2048) : ((MODE == EPI_PATCH || MODE == EPI_COS) ? 0 : 4096);
   static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
   static constexpr int OFF_BAR = OFF_EPI + GEMM_EPI_WARPS * EPI_WARP_BYTES;
   static constexpr int BAR_BYTES = 512;
@@ -108,14 +119,15 @@ __device__ __forceinline__ void chunk_mean_m2(const float (&v)[32], float& mean,
   m2 = (q0 + q1) + (q2 + q3);
 }
 
-// Affine epilogue of one 32-column chunk for BIAS / LNFOLD: v <- act(rstd * v - rstd * mu * c + b),
-// two columns per packed f32x2 instruction.
+// Affine epilogue of one 32-column chunk for BIAS / LNFOLD: v <- act(rstd * v + shift * c + b)
+// with shift = rstd * (ctr - mean) (the accumulator holds bf16(x - ctr) . W_gamma), two columns
+// per packed f32x2 instruction.
 template <int MODE>
-__device__ __forceinline__ void epi_affine(const EpiParams& ep, float (&v)[32], int n, float mu, float rstd) {
+__device__ __forceinline__ void epi_affine(const EpiParams& ep, float (&v)[32], int n, float shift, float rstd) {
   const float4* b4 = reinterpret_cast<const float4*>(ep.bias + n);
   if (MODE == EPI_LNFOLD) {
     const float4* c4 = reinterpret_cast<const float4*>(ep.colsum + n);
-    const float2 nrm = make_float2(-rstd * mu, -rstd * mu);
+    const float2 nrm = make_float2(shift, shift);
     const float2 rs = make_float2(rstd, rstd);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -152,9 +164,9 @@ __device__ __forceinline__ void epi_affine(const EpiParams& ep, float (&v)[32], 
   }
 }
 
-// LNFOLD: the row's LayerNorm mean and 1 / std, rebuilt from the producer's partial (mean, M2)
-// pairs (merged in column order); the loads go out eight at a time so their latencies overlap.
-__device__ __forceinline__ void lnfold_row_stats(const EpiParams& ep, int row, float& mu, float& rstd) {
+// The row's mean and sum of squared deviations, merged from the producer's partial (mean, M2)
+// pairs in column order; the loads go out eight at a time so their latencies overlap.
+__device__ __forceinline__ void merge_row_stats(const EpiParams& ep, int row, float& mu, float& m2out) {
   float n = 0.f, mean = 0.f, m2 = 0.f;
   const float2* s = ep.stats_in + static_cast<size_t>(row) * ep.nt;
   for (int t0 = 0; t0 < ep.nt; t0 += 8) {
@@ -166,7 +178,16 @@ __device__ __forceinline__ void lnfold_row_stats(const EpiParams& ep, int row, f
       if (t0 + u < ep.nt) merge_stats(n, mean, m2, static_cast<float>(ep.nt_cols), st[u].x, st[u].y);
   }
   mu = mean;
+  m2out = m2;
+}
+
+// LNFOLD: rstd of the row and the shift rstd * (ctr - mean) that turns the accumulator of the
+// re-centred operand into the accumulator of x - mean.
+__device__ __forceinline__ void lnfold_row_stats(const EpiParams& ep, int row, float& shift, float& rstd) {
+  float mu, m2;
+  merge_row_stats(ep, row, mu, m2);
   rstd = rsqrtf(m2 / static_cast<float>(ep.D) + ep.eps);
+  shift = rstd * (ep.ctr[row] - mu);
 }
 
 // Pulls the 128-byte lines of v[n0 .. n0 + cols - 1] (cols a multiple of 32) into L1, so that
@@ -179,10 +200,18 @@ __device__ __forceinline__ void prefetch_cols_l1(const float* v, int n0, int col
 // Work a BIAS / LNFOLD epilogue warp does before it waits for its accumulator: the rows'
 // LayerNorm statistics (LNFOLD) and the columns' bias / colsum lines.  (The same prefetch in the
 // residual epilogue, whose x loads already run a chunk ahead, measured 1-2 % slower.)
+//
+// RESID: the centre of the row's new bf16 copy, the mean of x before this update (merged from
+// stats_in), returned in `mu`.  Every CTA that writes a part of the row computes the same value.
 template <int BN, int MODE>
 __device__ __forceinline__ void epilogue_prologue(const EpiParams& ep, int row, int n0, float& mu, float& rstd) {
   mu = 0.f;
   rstd = 0.f;
+  if (MODE == EPI_RESID) {
+    float m2;
+    if (row < ep.M) merge_row_stats(ep, row, mu, m2);
+    return;
+  }
   if (MODE != EPI_BIAS && MODE != EPI_LNFOLD) return;
   prefetch_cols_l1(ep.bias, n0, BN / 2);
   if (MODE == EPI_LNFOLD) prefetch_cols_l1(ep.colsum, n0, BN / 2);
@@ -192,7 +221,7 @@ __device__ __forceinline__ void epilogue_prologue(const EpiParams& ep, int row, 
 // BIAS / LNFOLD: one warp's half of a tile (rows row0 .. row0 + 31, columns n0 .. n0 + BN/2 - 1),
 // 64 columns per TMA store from the warp's staging buffer `obuf` (32 rows x 128 bytes, 128B
 // swizzle: 16-byte chunk k of row r sits at chunk k ^ (r % 8)).  mu / rstd: this thread's row
-// statistics (LNFOLD).
+// statistics (LNFOLD: mu carries the centre shift of lnfold_row_stats).
 template <int BN, int MODE>
 __device__ __forceinline__ void epilogue_store_bf16(const EpiParams& ep, const CUtensorMap* tmO, uint32_t taddr,
                                                     int row0, int n0, uint8_t* obuf, float mu, float rstd) {
@@ -229,17 +258,23 @@ __device__ __forceinline__ void epilogue_store_bf16(const EpiParams& ep, const C
 
 // RESID: one warp's half of a tile.  x arrives by TMA into xbuf[c & 1] (32 rows x 128 bytes, 128B
 // swizzle), chunk c + 1 is requested while chunk c is processed; the updated x goes back into the
-// same buffer and, with its bf16 copy (xbbuf: 32 rows x 64 bytes, 64B swizzle), out by TMA stores.
-// Row statistics (mean, M2) are written per row for each group of ep.stats_cols columns.
+// same buffer and, with its re-centred bf16 copy bf16(x - centre) (xbbuf: 32 rows x 64 bytes, 64B
+// swizzle), out by TMA stores.  `centre` is this thread's row's mean of x before the update (the
+// same value in every CTA that writes a part of the row); the warps of column group 0 record it
+// in ep.ctr for the folded LayerNorm that reads the copy.  Row statistics (mean, M2) of the new x
+// are written per row for each group of ep.stats_cols columns.
 template <int BN>
 __device__ __forceinline__ void epilogue_resid(const EpiParams& ep, const CUtensorMap* tmX, const CUtensorMap* tmXb,
-                                               uint32_t taddr, int row0, int n0, uint8_t* xbuf0, uint8_t* xbbuf,
-                                               uint64_t* xfull, uint32_t (&xph)[2], bool (&xpending)[2],
-                                               volatile int* abort_flag, int* gstatus, bool& ok) {
+                                               uint32_t taddr, int row0, int n0, float centre, uint8_t* xbuf0,
+                                               uint8_t* xbbuf, uint64_t* xfull, uint32_t (&xph)[2],
+                                               bool (&xpending)[2], volatile int* abort_flag, int* gstatus, bool& ok) {
   constexpr int HALF = BN / 2;
   constexpr int CHUNKS = HALF / 32;
   const int lane = threadIdx.x & 31;
   const int row = row0 + lane;
+  if (n0 == 0 && row < ep.M) ep.ctr[row] = centre;
+  const float2 nc = make_float2(-centre, -centre);
+  const unsigned long long wlim = wait_limit(ep.wait_ns);
   float run_n = 0.f, run_mean = 0.f, run_m2 = 0.f;
 #pragma unroll 1
   for (int c = 0; c < CHUNKS; ++c) {
@@ -254,7 +289,7 @@ __device__ __forceinline__ void epilogue_resid(const EpiParams& ep, const CUtens
       }
     }
     __syncwarp();
-    if (!mbar_wait(&xfull[buf], xph[buf], abort_flag, gstatus, DEV_TIMEOUT_GEMM + 6)) {
+    if (!mbar_wait(&xfull[buf], xph[buf], abort_flag, gstatus, DEV_TIMEOUT_GEMM + 6, wlim)) {
       ok = false;
       return;
     }
@@ -291,11 +326,15 @@ __device__ __forceinline__ void epilogue_resid(const EpiParams& ep, const CUtens
           make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
+      const float2 c0 = fadd2(make_float2(v[8 * k + 0], v[8 * k + 1]), nc);
+      const float2 c1 = fadd2(make_float2(v[8 * k + 2], v[8 * k + 3]), nc);
+      const float2 c2 = fadd2(make_float2(v[8 * k + 4], v[8 * k + 5]), nc);
+      const float2 c3 = fadd2(make_float2(v[8 * k + 6], v[8 * k + 7]), nc);
       uint4 w;
-      w.x = pack_bf16x2(v[8 * k + 0], v[8 * k + 1]);
-      w.y = pack_bf16x2(v[8 * k + 2], v[8 * k + 3]);
-      w.z = pack_bf16x2(v[8 * k + 4], v[8 * k + 5]);
-      w.w = pack_bf16x2(v[8 * k + 6], v[8 * k + 7]);
+      w.x = pack_bf16x2(c0.x, c0.y);
+      w.y = pack_bf16x2(c1.x, c1.y);
+      w.z = pack_bf16x2(c2.x, c2.y);
+      w.w = pack_bf16x2(c3.x, c3.y);
       *reinterpret_cast<uint4*>(xbbuf + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) = w;
     }
     fence_proxy_async_smem();
@@ -319,7 +358,9 @@ __device__ __forceinline__ void epilogue_resid(const EpiParams& ep, const CUtens
   }
 }
 
-// PATCH: rows of the GEMM are scattered to token rows, so this epilogue writes directly.
+// PATCH: rows of the GEMM are scattered to token rows, so this epilogue writes x directly
+// (x[b * T + 1 + R + p] = acc + bias + pos[p]); the bf16 copy, its centre and the row statistics
+// follow in token_prep_kernel, which sees whole rows.
 template <int BN>
 __device__ __forceinline__ void epilogue_patch(const EpiParams& ep, uint32_t taddr, int row, int n0) {
   constexpr int HALF = BN / 2;
@@ -332,7 +373,6 @@ __device__ __forceinline__ void epilogue_patch(const EpiParams& ep, uint32_t tad
     xrow = b * ep.T + 1 + ep.R + p;
     posrow = ep.pos + static_cast<size_t>(p + ep.pos_off) * ep.N;
   }
-  float run_n = 0.f, run_mean = 0.f, run_m2 = 0.f;
 #pragma unroll 1
   for (int c = 0; c < HALF / 32; ++c) {
     float v[32];
@@ -354,30 +394,35 @@ __device__ __forceinline__ void epilogue_patch(const EpiParams& ep, uint32_t tad
       float4* xp = reinterpret_cast<float4*>(ep.x + static_cast<size_t>(xrow) * ep.N + n);
 #pragma unroll
       for (int j = 0; j < 8; ++j) xp[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-      uint4* o = reinterpret_cast<uint4*>(ep.xb + static_cast<size_t>(xrow) * ep.N + n);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint4 w;
-        w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-        w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-        w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-        w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-        o[j] = w;
-      }
-      float s = 0.f;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) s += v[j];
-      const float cm = s * (1.0f / 32.0f);
-      float q = 0.f;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float d = v[j] - cm;
-        q = fmaf(d, d, q);
-      }
-      merge_stats(run_n, run_mean, run_m2, 32.f, cm, q);
     }
   }
-  if (valid) ep.stats_out[static_cast<size_t>(xrow) * (ep.N / HALF) + n0 / HALF] = make_float2(run_mean, run_m2);
+}
+
+// COS: the patch-text cosine map.  Row m = w * P + p of the GEMM (window w, patch p), column c
+// (class) goes to cos[(w * ncls + c) * P + p]: for each column the 32 lanes of a warp write 32
+// consecutive patches of one class row (128-byte segments).  Padding columns are skipped.
+template <int BN>
+__device__ __forceinline__ void epilogue_cos(const EpiParams& ep, uint32_t taddr, int row, int n0) {
+  constexpr int HALF = BN / 2;
+  float* base = nullptr;
+  if (row < ep.M) {
+    const int w = row / ep.P;
+    const int p = row - w * ep.P;
+    base = ep.cos + static_cast<size_t>(w) * ep.ncls * ep.P + p;
+  }
+#pragma unroll 1
+  for (int c = 0; c < HALF / 32; ++c) {
+    const int n = n0 + c * 32;
+    if (n >= ep.ncls) break;  // warp-uniform: the rest of this half is padding
+    float v[32];
+    __syncwarp();
+    tmem_ld32(taddr + c * 32, v);
+    if (base != nullptr) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (n + j < ep.ncls) base[static_cast<size_t>(n + j) * ep.P] = v[j];
+    }
+  }
 }
 
 // tmO1 / tmO2: BIAS / LNFOLD -> tmO1 = output [M, ldo] bf16 (box 64 x 32, 128B swizzle);
@@ -390,6 +435,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                         int N, int K, EpiParams ep, int* gstatus) {
   using Cfg = GemmCfg<BN, MODE>;
   constexpr int STAGES = Cfg::STAGES;
+  const unsigned long long wlim = wait_limit(ep.wait_ns);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -422,7 +468,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (MODE != EPI_PATCH) tma_prefetch_desc(&tmO1);
+    if (MODE != EPI_PATCH && MODE != EPI_COS) tma_prefetch_desc(&tmO1);
     if (MODE == EPI_RESID) tma_prefetch_desc(&tmO2);
   }
   if (warp == 1) {
@@ -452,7 +498,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int nb = tile - mb * num_n;
       bool ok = true;
       for (int kb = 0; kb < KB; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 1)) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 1, wlim)) {
           ok = false;
           break;
         }
@@ -482,11 +528,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 2)) break;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 2, wlim)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 3)) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 3, wlim)) {
             ok = false;
             break;
           }
@@ -538,17 +584,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       float mu, rstd;
       epilogue_prologue<BN, MODE>(ep, row0 + lane, n0, mu, rstd);
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 4)) break;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 4, wlim)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + half * (BN / 2));
       __syncwarp();
       if (MODE == EPI_RESID) {
-        epilogue_resid<BN>(ep, &tmO1, &tmO2, taddr, row0, n0, wbuf, wbuf + 8192, wxfull, xph, xpending, abort_flag,
+        epilogue_resid<BN>(ep, &tmO1, &tmO2, taddr, row0, n0, mu, wbuf, wbuf + 8192, wxfull, xph, xpending, abort_flag,
                            gstatus, ok);
         if (!ok) break;
       } else if (MODE == EPI_PATCH) {
         epilogue_patch<BN>(ep, taddr, row0 + lane, n0);
+      } else if (MODE == EPI_COS) {
+        epilogue_cos<BN>(ep, taddr, row0 + lane, n0);
       } else {
         epilogue_store_bf16<BN, MODE>(ep, &tmO1, taddr, row0, n0, wbuf, mu, rstd);
       }
@@ -606,7 +654,7 @@ struct PairCfg {
   static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(MODE != EPI_PATCH, "the patch GEMM runs unpaired");
+  static_assert(MODE != EPI_PATCH && MODE != EPI_COS, "the patch and cosine GEMMs run unpaired");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(8 * (2 * STAGES + 5 + 2 * GEMM_EPI_WARPS) + 8 <= BAR_BYTES, "barrier area");
 };
@@ -633,6 +681,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   using Cfg = PairCfg<MODE>;
   constexpr int BN = Cfg::BN;
   constexpr int STAGES = Cfg::STAGES;
+  const unsigned long long wlim = wait_limit(ep.wait_ns);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -704,7 +753,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       const int nb = tile - mb * num_n;
       bool ok = true;
       for (int kb = 0; kb < KB; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 5)) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 5, wlim)) {
           ok = false;
           break;
         }
@@ -742,11 +791,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = cid; tile < num_tiles && ok; tile += ncl) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 6)) break;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 6, wlim)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 7)) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 7, wlim)) {
             ok = false;
             break;
           }
@@ -798,13 +847,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       }
       float mu = 0.f, rstd = 0.f;
       if (active) epilogue_prologue<BN, MODE>(ep, row0 + lane, n0, mu, rstd);
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 8)) break;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, gstatus, DEV_TIMEOUT_GEMM + 8, wlim)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + half * (BN / 2));
       __syncwarp();
       if (MODE == EPI_RESID && active) {
-        epilogue_resid<BN>(ep, &tmO1, &tmO2, taddr, row0, n0, wbuf, wbuf + 8192, wxfull, xph, xpending, abort_flag,
+        epilogue_resid<BN>(ep, &tmO1, &tmO2, taddr, row0, n0, mu, wbuf, wbuf + 8192, wxfull, xph, xpending, abort_flag,
                            gstatus, ok);
         if (!ok) break;
       } else if (MODE != EPI_RESID && active) {

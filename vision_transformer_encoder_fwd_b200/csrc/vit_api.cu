@@ -2,7 +2,8 @@
 //
 // Plans and launches the encoder forward of the DINOv2/DINOv3 ViT ("DINOv2 n semantic"
 // diagram; kornia/dinov3 card) and the dino.txt zero-shot scoring on one B200:
-//   im2col -> patch GEMM (+bias +pos, token placement, row stats) -> CLS/register rows
+//   im2col -> patch GEMM (+bias +pos, token placement) -> CLS/register rows, row stats and the
+//   re-centred bf16 copy of every token row
 //   per block: QKV GEMM (LayerNorm folded) -> attention -> proj GEMM (+LS, residual, stats)
 //              -> FC1 GEMM (LayerNorm folded, GELU) -> FC2 GEMM (+LS, residual, stats) [-> tap]
 //   final LayerNorm -> descriptor / patch tokens
@@ -10,6 +11,7 @@
 // workspace, encodes TMA descriptors and enqueues launches.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -235,7 +237,7 @@ cudaError_t launch_gemm_pair_t(const CUtensorMap& a, const CUtensorMap& b, const
 }
 
 // o1 / o2: BIAS, LNFOLD: o1 = bf16 output map (tmap_out_bf16); RESID: o1 = x (tmap_x_f32),
-// o2 = xb (tmap_xb_bf16); PATCH: not read (any valid map).  bn: 128 or 256 (one CTA per tile,
+// o2 = xb (tmap_xb_bf16); PATCH, COS: not read (any valid map).  bn: 128 or 256 (one CTA per tile,
 // B map boxes of bn rows) or BN_PAIR (B map boxes of 128 rows; not for PATCH).
 cudaError_t launch_gemm(int bn, int mode, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o1,
                         const CUtensorMap& o2, int M, int N, int K, const EpiParams& ep, int* st, cudaStream_t s,
@@ -260,18 +262,19 @@ cudaError_t launch_gemm(int bn, int mode, const CUtensorMap& a, const CUtensorMa
     case EPI_BIAS: return launch_gemm_t<128, EPI_BIAS>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
     case EPI_LNFOLD: return launch_gemm_t<128, EPI_LNFOLD>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
     case EPI_RESID: return launch_gemm_t<128, EPI_RESID>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
+    case EPI_COS: return launch_gemm_t<128, EPI_COS>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
     default: return launch_gemm_t<128, EPI_PATCH>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
   }
 }
 
 cudaError_t launch_attention(const CUtensorMap& tm, const __nv_bfloat16* qkv, int B, int T, int heads,
-                             __nv_bfloat16* out, int* st, cudaStream_t s) {
+                             __nv_bfloat16* out, int* st, cudaStream_t s, unsigned long long wait_ns) {
   static std::atomic<uint64_t> attr_done{0};
   cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel, AttnCfg::SMEM_BYTES, attr_done);
   if (e != cudaSuccess) return e;
   const int n_qtiles = (T + ATT_BM - 1) / ATT_BM;
   dim3 grid((n_qtiles + ATT_NT - 1) / ATT_NT, heads, B);
-  attn_fwd_tc_kernel<<<grid, ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, qkv, T, heads * 64, out, st);
+  attn_fwd_tc_kernel<<<grid, ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, qkv, T, heads * 64, out, st, wait_ns);
   return cudaGetLastError();
 }
 
@@ -344,6 +347,7 @@ struct vit_model {
     float *pred_w = nullptr, *pred_b = nullptr, *zero = nullptr;
   } dense;  // dense head on the taps (vit_set_dense_head)
   int* d_status = nullptr;
+  unsigned long long wait_ns = 0;  // pipeline-wait limit of this model's launches (0: 2 s)
   int last_launches = 0;
   std::vector<void*> allocs;
   // per-launch profiling (vit_profile_begin / vit_profile_end)
@@ -356,7 +360,7 @@ struct vit_model {
 namespace {
 
 struct WsLayout {
-  size_t x, xb, stats, attn, big, pos, total;
+  size_t x, xb, stats, ctr, attn, big, pos, total;
 };
 
 // The token geometry of one forward: input H x W, patch grid gh x gw (the convolution's
@@ -403,8 +407,12 @@ WsLayout ws_layout(const vit_model* m, int B, const Geom& g) {
   off = align_up(off + M * D * 4, 1024);
   L.xb = off;
   off = align_up(off + M * D * 2, 1024);
+  // two statistics buffers: a residual GEMM reads the partials of x before its update (the centre
+  // of the new bf16 copy) from one and writes those of the new x into the other
   L.stats = off;
-  off = align_up(off + M * m->nt * 8, 1024);
+  off = align_up(off + 2 * M * m->nt * 8, 1024);
+  L.ctr = off;
+  off = align_up(off + M * 4, 1024);
   L.attn = off;
   off = align_up(off + M * D * 2, 1024);
   L.big = off;
@@ -415,8 +423,17 @@ WsLayout ws_layout(const vit_model* m, int B, const Geom& g) {
   return L;
 }
 
-// Profiling brackets around one launch (no-ops unless profiling is on and capacity remains).
+// NVTX range names of the launch kinds (the VIT_K_* order of vit.h).
+const char* const kKindName[VIT_K_COUNT] = {
+    "vit/im2col",   "vit/patch_gemm", "vit/token_prep",  "vit/qkv_gemm", "vit/attention",  "vit/proj_gemm",
+    "vit/fc1_gemm", "vit/fc2_gemm",   "vit/tap",         "vit/final_ln", "vit/seg_split",  "vit/seg_cos_gemm",
+    "vit/seg_map",  "vit/pos_resize", "vit/head_tokens", "vit/dense_gemm", "vit/dense_aux"};
+
+// Brackets around one launch: an NVTX range named after the launch kind (seen by Nsight tools
+// when one is attached, a no-op otherwise) and, while per-launch profiling is on and capacity
+// remains, two CUDA events on the launch stream.
 int prof_open(vit_model* m, int kind, cudaStream_t s) {
+  nvtxRangePushA(kKindName[kind]);
   if (!m->prof_on || m->prof_used >= static_cast<int>(m->prof_kind.size())) return -1;
   const int slot = m->prof_used++;
   m->prof_kind[slot] = kind;
@@ -425,6 +442,20 @@ int prof_open(vit_model* m, int kind, cudaStream_t s) {
 }
 void prof_close(vit_model* m, int slot, cudaStream_t s) {
   if (slot >= 0) cudaEventRecord(m->prof_ev[2 * slot + 1], s);
+  nvtxRangePop();
+}
+
+// Every launch of a model must run on the device whose memory holds its weights, derived
+// copies and TMA descriptors; the caller picks the current device, so each entry point that
+// launches checks it before anything is enqueued.
+vit_status check_device(const vit_model* m, const char* fn) {
+  int cur = 0;
+  CK(cudaGetDevice(&cur));
+  if (cur != m->device) {
+    set_err("%s called with device %d current; the model lives on device %d", fn, cur, m->device);
+    return VIT_E_INVALID_ARG;
+  }
+  return VIT_OK;
 }
 
 vit_status alloc_dev(vit_model* m, void** p, size_t bytes) {
@@ -524,7 +555,8 @@ vit_status build_block(vit_model* m, const vit_block_weights& src, BlockW& b, cu
 struct Scratch {
   float* x;
   __nv_bfloat16* xb;
-  float2* stats;
+  float2* stats[2];
+  float* ctr;
   __nv_bfloat16* attn;
   __nv_bfloat16* big;
 };
@@ -535,7 +567,9 @@ struct Scratch {
 vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, const vit_outputs* out, void* ws,
                        size_t ws_bytes, cudaStream_t s, bool head = false, __nv_bfloat16* tap_rows = nullptr) {
   const vit_config& c = m->cfg;
-  vit_status gst = check_geom(m, B, g);
+  vit_status gst = check_device(m, "the forward");
+  if (gst != VIT_OK) return gst;
+  gst = check_geom(m, B, g);
   if (gst != VIT_OK) return gst;
   const WsLayout L = ws_layout(m, B, g);
   if (ws == nullptr || ws_bytes < L.total) {
@@ -547,11 +581,16 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
     return VIT_E_INVALID_ARG;
   }
   uint8_t* w8 = static_cast<uint8_t*>(ws);
-  Scratch S{reinterpret_cast<float*>(w8 + L.x), reinterpret_cast<__nv_bfloat16*>(w8 + L.xb),
-            reinterpret_cast<float2*>(w8 + L.stats), reinterpret_cast<__nv_bfloat16*>(w8 + L.attn),
-            reinterpret_cast<__nv_bfloat16*>(w8 + L.big)};
   const int D = c.dim, F = c.mlp_dim, T = g.T, P = g.P, R = c.n_registers;
   const int M = B * T, Mp = B * P;
+  Scratch S{reinterpret_cast<float*>(w8 + L.x),
+            reinterpret_cast<__nv_bfloat16*>(w8 + L.xb),
+            {reinterpret_cast<float2*>(w8 + L.stats),
+             reinterpret_cast<float2*>(w8 + L.stats) + static_cast<size_t>(M) * m->nt},
+            reinterpret_cast<float*>(w8 + L.ctr),
+            reinterpret_cast<__nv_bfloat16*>(w8 + L.attn),
+            reinterpret_cast<__nv_bfloat16*>(w8 + L.big)};
+  int cur = 0;  // S.stats[cur] holds the partial statistics of the current x
   int launches = 0;
   const float* pos = m->pos;
   if (!g.native) {
@@ -583,12 +622,11 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
   ++launches;
   {
     EpiParams ep{};
+    ep.wait_ns = m->wait_ns;
     ep.M = Mp;
     ep.N = D;
     ep.bias = m->patch_b;
     ep.x = S.x;
-    ep.xb = S.xb;
-    ep.stats_out = S.stats;
     ep.pos = pos;
     ep.P = P;
     ep.T = T;
@@ -600,8 +638,8 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
     ++launches;
   }
   { const int ps_ = prof_open(m, VIT_K_PREFIX, s);
-  prefix_tokens_kernel<<<dim3(m->nt, 1 + R, B), 32, 0, s>>>(m->cls, m->reg, pos, c.pos_on_cls, T, D, m->stats_cols,
-                                                             S.x, S.xb, S.stats);
+  token_prep_kernel<<<(M + 7) / 8, 256, 0, s>>>(m->cls, m->reg, pos, c.pos_on_cls, M, T, R, D, m->stats_cols, S.x,
+                                                 S.xb, S.stats[cur], S.ctr);
   prof_close(m, ps_, s); }
   CKL();
   ++launches;
@@ -613,11 +651,13 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
     {
       const int bn = pick_bn(M, 3 * D, m->nsm);
       EpiParams ep{};
+      ep.wait_ns = m->wait_ns;
       ep.M = M;
       ep.N = 3 * D;
       ep.bias = bw.qkv_b;
       ep.colsum = bw.qkv_c;
-      ep.stats_in = S.stats;
+      ep.stats_in = S.stats[cur];
+      ep.ctr = S.ctr;
       ep.nt = m->nt;
       ep.nt_cols = m->stats_cols;
       ep.D = D;
@@ -630,19 +670,24 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
       ++launches;
     }
     { const int ps_ = prof_open(m, VIT_K_ATTENTION, s);
-    CK(launch_attention(tm_qkv3, S.big, B, T, c.heads, S.attn, m->d_status, s));
+    CK(launch_attention(tm_qkv3, S.big, B, T, c.heads, S.attn, m->d_status, s, m->wait_ns));
     prof_close(m, ps_, s); }
     ++launches;
     // proj + layer scale + residual
     {
       EpiParams ep{};
+      ep.wait_ns = m->wait_ns;
       ep.M = M;
       ep.N = D;
       ep.bias = bw.proj_b;
       ep.ls = bw.ls1;
       ep.x = S.x;
       ep.xb = S.xb;
-      ep.stats_out = S.stats;
+      ep.ctr = S.ctr;
+      ep.stats_in = S.stats[cur];
+      ep.nt = m->nt;
+      ep.nt_cols = m->stats_cols;
+      ep.stats_out = S.stats[cur ^ 1];
       ep.stats_cols = m->stats_cols;
       const int bnr = pick_bn_res(M, D, m->bn_res, m->nsm);
       { const int ps_ = prof_open(m, VIT_K_PROJ_GEMM, s);
@@ -650,16 +695,19 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
                      m->d_status, s, m->nsm));
       prof_close(m, ps_, s); }
       ++launches;
+      cur ^= 1;
     }
     // LN2 (folded) + FC1 + GELU
     {
       const int bn = pick_bn(M, F, m->nsm);
       EpiParams ep{};
+      ep.wait_ns = m->wait_ns;
       ep.M = M;
       ep.N = F;
       ep.bias = bw.fc1_b;
       ep.colsum = bw.fc1_c;
-      ep.stats_in = S.stats;
+      ep.stats_in = S.stats[cur];
+      ep.ctr = S.ctr;
       ep.nt = m->nt;
       ep.nt_cols = m->stats_cols;
       ep.D = D;
@@ -675,13 +723,18 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
     // FC2 + layer scale + residual
     {
       EpiParams ep{};
+      ep.wait_ns = m->wait_ns;
       ep.M = M;
       ep.N = D;
       ep.bias = bw.fc2_b;
       ep.ls = bw.ls2;
       ep.x = S.x;
       ep.xb = S.xb;
-      ep.stats_out = S.stats;
+      ep.ctr = S.ctr;
+      ep.stats_in = S.stats[cur];
+      ep.nt = m->nt;
+      ep.nt_cols = m->stats_cols;
+      ep.stats_out = S.stats[cur ^ 1];
       ep.stats_cols = m->stats_cols;
       const int bnr = pick_bn_res(M, D, m->bn_res, m->nsm);
       { const int ps_ = prof_open(m, VIT_K_FC2_GEMM, s);
@@ -689,6 +742,7 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
                      m->d_status, s, m->nsm));
       prof_close(m, ps_, s); }
       ++launches;
+      cur ^= 1;
     }
     return VIT_OK;
   };
@@ -726,7 +780,8 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
     const long long rows = static_cast<long long>(M);
     { const int ps_ = prof_open(m, VIT_K_FINAL_LN, s);
     final_ln_stream_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(S.x, m->norm_w, m->norm_b, rows, D, c.ln_eps,
-                                                                          m->stats_cols, S.xb, S.stats, m->d_status + 1);
+                                                                          m->stats_cols, S.xb, S.stats[cur], S.ctr,
+                                                                          m->d_status + 1);
     prof_close(m, ps_, s); }
     CKL();
     ++launches;
@@ -771,6 +826,9 @@ vit_status check_outputs(const vit_outputs* out) {
 }
 
 }  // namespace
+
+// defined with the allocation-free forward at the end of this file
+vit_status noalloc_resolve(int dev);
 
 // ------------------------------------------------------------------ C ABI
 extern "C" {
@@ -860,7 +918,9 @@ vit_status vit_create(const vit_config* cfg, const vit_weights* w, vit_model** o
       if ((e = build_block(m, w->blocks[l], m->blocks[l], s)) != VIT_OK) return e;
     }
     CK(cudaStreamSynchronize(s));
-    return VIT_OK;
+    // the allocation-free forward's scratch address on this device, looked up now, outside
+    // any stream capture a caller might start later
+    return noalloc_resolve(m->device);
   };
   st = run();
   cudaStreamDestroy(s);
@@ -1068,6 +1128,7 @@ static vit_status run_dense(vit_model* m, const float* images, int B, const Geom
         !tmap_out_bf16(&to, out, N, Mp, N))
       return VIT_E_CUDA;
     EpiParams ep{};
+    ep.wait_ns = m->wait_ns;
     ep.M = static_cast<int>(Mp);
     ep.N = N;
     ep.bias = bias;
@@ -1297,6 +1358,8 @@ vit_status vit_forward_host(vit_model* m, const float* images_host, int32_t B, f
     set_err("host-path workspace must be >= %zu bytes and 256-byte aligned", need);
     return VIT_E_WORKSPACE;
   }
+  st = check_device(m, "vit_forward_host");
+  if (st != VIT_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t img_b = static_cast<size_t>(B) * 3 * m->cfg.img_h * m->cfg.img_w * 4;
   const size_t img = align_up(img_b, 1024);
@@ -1365,9 +1428,16 @@ static vit_status seg_plan(const vit_model* m, int32_t H, int32_t W, int32_t C, 
   return check_geom(m, nwin, p->g);
 }
 
+// Classes padded to the GEMM's column tile for the cosine map.
+static int seg_cpad(int C) { return (C + 127) / 128 * 128; }
+
+// Scoring scratch ahead of the encoder's workspace: fp32 tokens [rows, D], the split operands
+// A3 [rows, 3D] and B3 [Cpad, 3D] (bf16) and the cosine map [windows, C, P] (fp32).
 static size_t seg_head_bytes(const vit_model* m, const SegPlan& p, int C) {
   const size_t rows = static_cast<size_t>(p.ny) * p.nx * p.g.P;
-  return align_up(rows * m->cfg.dim * 4, 1024) + align_up(rows * 4, 1024) + align_up(rows * C * 4, 1024);
+  const size_t D = m->cfg.dim;
+  return align_up(rows * D * 4, 1024) + align_up(rows * 3 * D * 2, 1024) +
+         align_up(static_cast<size_t>(seg_cpad(C)) * 3 * D * 2, 1024) + align_up(rows * C * 4, 1024);
 }
 
 vit_status vit_seg_workspace_size(const vit_model* m, int32_t H, int32_t W, int32_t C, int32_t mode, int32_t side,
@@ -1403,10 +1473,13 @@ vit_status vit_seg_zero_shot(vit_model* m, const float* image, int32_t H, int32_
   const int ny = plan.ny, nx = plan.nx, nwin = ny * nx, P = plan.g.P;
   const size_t rows = static_cast<size_t>(nwin) * P;
   uint8_t* w8 = static_cast<uint8_t*>(ws);
+  const int D = c.dim, Cpad = seg_cpad(C);
   float* tok = reinterpret_cast<float*>(w8);
-  size_t off = align_up(rows * c.dim * 4, 1024);
-  float* inv = reinterpret_cast<float*>(w8 + off);
-  off += align_up(rows * 4, 1024);
+  size_t off = align_up(rows * D * 4, 1024);
+  __nv_bfloat16* a3 = reinterpret_cast<__nv_bfloat16*>(w8 + off);
+  off += align_up(rows * 3 * D * 2, 1024);
+  __nv_bfloat16* b3 = reinterpret_cast<__nv_bfloat16*>(w8 + off);
+  off += align_up(static_cast<size_t>(Cpad) * 3 * D * 2, 1024);
   float* cosm = reinterpret_cast<float*>(w8 + off);
   off += align_up(rows * C * 4, 1024);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -1419,16 +1492,28 @@ vit_status vit_seg_zero_shot(vit_model* m, const float* image, int32_t H, int32_
   st = run_forward(m, src, nwin, plan.g, &o, w8 + off, ws_bytes - off, s, /*head=*/true);
   if (st != VIT_OK) return st;
   int launches = m->last_launches;
+  // the cosine map on the tensor cores: split operands, then A3 . B3^T scattered to [w, c, p]
   { const int ps_ = prof_open(m, VIT_K_SEG_NORM, s);
-  token_inv_norm_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(tok, static_cast<long long>(rows), c.dim, inv);
+  cos_split_tokens_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(tok, static_cast<long long>(rows), D, a3);
+  cos_split_text_kernel<<<(Cpad + 7) / 8, 256, 0, s>>>(text, C, Cpad, D, b3);
   prof_close(m, ps_, s); }
   CKL();
-  dim3 cg(static_cast<unsigned>((rows + 63) / 64), static_cast<unsigned>((C + 63) / 64));
-  { const int ps_ = prof_open(m, VIT_K_SEG_COS, s);
-  cos_gemm_kernel<<<cg, 256, 0, s>>>(tok, inv, text, P, static_cast<long long>(rows), C, c.dim, cosm);
-  prof_close(m, ps_, s); }
-  CKL();
-  launches += 2;
+  {
+    CUtensorMap ta, tb;
+    if (!tmap_2d(&ta, a3, 3 * D, rows, 3 * D, 64, GEMM_BM) || !tmap_2d(&tb, b3, 3 * D, Cpad, 3 * D, 64, 128))
+      return VIT_E_CUDA;
+    EpiParams ep{};
+    ep.wait_ns = m->wait_ns;
+    ep.M = static_cast<int>(rows);
+    ep.N = Cpad;
+    ep.P = P;
+    ep.cos = cosm;
+    ep.ncls = C;
+    { const int ps_ = prof_open(m, VIT_K_SEG_COS, s);
+    CK(launch_gemm(128, EPI_COS, ta, tb, ta, ta, static_cast<int>(rows), Cpad, 3 * D, ep, m->d_status, s, m->nsm));
+    prof_close(m, ps_, s); }
+  }
+  launches += 3;
   const long long pix = static_cast<long long>(H) * W;
   if (mode == VIT_SEG_SLIDE) {
     // the tiled kernel when every 16 x 16 tile meets at most SLIDE_TILE_WIN windows, the classes fit
@@ -1491,6 +1576,15 @@ vit_status vit_poll(vit_model* m, vit_stream_t stream) {
   return VIT_OK;
 }
 
+vit_status vit_set_wait_limit(vit_model* m, uint64_t ns) {
+  if (!m) {
+    set_err("model is NULL");
+    return VIT_E_INVALID_ARG;
+  }
+  m->wait_ns = ns;
+  return VIT_OK;
+}
+
 int32_t vit_last_launch_count(const vit_model* m) { return m ? m->last_launches : 0; }
 
 vit_status vit_profile_begin(vit_model* m, int32_t capacity) {
@@ -1535,8 +1629,9 @@ vit_status vit_profile_end(vit_model* m, float* total_ms, int32_t* launches) {
 }
 
 // ------------------------------------------------------------------ stage entry points
-vit_status vit_stage_linear(const void* A, const void* W, const float* bias, int32_t M, int32_t N, int32_t K,
-                            int32_t gelu, void* out, int32_t* status, vit_stream_t stream) {
+vit_status vit_stage_linear_bounded(const void* A, const void* W, const float* bias, int32_t M, int32_t N, int32_t K,
+                                    int32_t gelu, void* out, int32_t* status, uint64_t wait_ns,
+                                    vit_stream_t stream) {
   if (!A || !W || !bias || !out || !status || !aligned16(A) || !aligned16(W) || !aligned16(bias) || !aligned16(out)) {
     set_err("NULL or misaligned pointer");
     return VIT_E_INVALID_ARG;
@@ -1559,12 +1654,18 @@ vit_status vit_stage_linear(const void* A, const void* W, const float* bias, int
   ep.bias = bias;
   ep.gelu = gelu;
   ep.ldo = N;
+  ep.wait_ns = wait_ns;
   CK(launch_gemm(bn, EPI_BIAS, ta, tb, to, to, M, N, K, ep, status, reinterpret_cast<cudaStream_t>(stream), nsm));
   return VIT_OK;
 }
 
-vit_status vit_stage_attention(const void* qkv, int32_t B, int32_t T, int32_t heads, void* out, int32_t* status,
-                               vit_stream_t stream) {
+vit_status vit_stage_linear(const void* A, const void* W, const float* bias, int32_t M, int32_t N, int32_t K,
+                            int32_t gelu, void* out, int32_t* status, vit_stream_t stream) {
+  return vit_stage_linear_bounded(A, W, bias, M, N, K, gelu, out, status, 0, stream);
+}
+
+vit_status vit_stage_attention_bounded(const void* qkv, int32_t B, int32_t T, int32_t heads, void* out,
+                                       int32_t* status, uint64_t wait_ns, vit_stream_t stream) {
   if (!qkv || !out || !status || !aligned16(qkv) || !aligned16(out)) {
     set_err("NULL or misaligned pointer");
     return VIT_E_INVALID_ARG;
@@ -1576,8 +1677,13 @@ vit_status vit_stage_attention(const void* qkv, int32_t B, int32_t T, int32_t he
   CUtensorMap tm;
   if (!tmap_qkv3d(&tm, qkv, B, T, heads * 64)) return VIT_E_CUDA;
   CK(launch_attention(tm, static_cast<const __nv_bfloat16*>(qkv), B, T, heads, static_cast<__nv_bfloat16*>(out), status,
-                      reinterpret_cast<cudaStream_t>(stream)));
+                      reinterpret_cast<cudaStream_t>(stream), wait_ns));
   return VIT_OK;
+}
+
+vit_status vit_stage_attention(const void* qkv, int32_t B, int32_t T, int32_t heads, void* out, int32_t* status,
+                               vit_stream_t stream) {
+  return vit_stage_attention_bounded(qkv, B, T, heads, out, status, 0, stream);
 }
 
 vit_status vit_stage_gelu(const float* x, int64_t n, float* y, vit_stream_t stream) {
@@ -1631,10 +1737,12 @@ namespace {
 // a stand-in and must never be handed to a kernel).
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[64] = {};
+}  // namespace
 
-vit_status noalloc_scratch(void** ptr) {
-  int dev = 0;
-  CK(cudaGetDevice(&dev));
+// Looks up the array's device address on the current device `dev` and caches it.  vit_create
+// calls this on the model's device, so a vit_forward_noalloc call (which requires that device to
+// be current) finds the address cached and never does the lookup itself, even under capture.
+vit_status noalloc_resolve(int dev) {
   if (dev < 0 || dev >= 64) {
     set_err("device index %d out of range for the fixed scratch table", dev);
     return VIT_E_UNSUPPORTED;
@@ -1645,7 +1753,33 @@ vit_status noalloc_scratch(void** ptr) {
     CK(cudaGetSymbolAddress(&p, g_noalloc_scratch));
     g_noalloc_ptr[dev] = p;
   }
-  *ptr = g_noalloc_ptr[dev];
+  return VIT_OK;
+}
+
+namespace {
+// The cached address for the model's device.  Should it be missing (it cannot be after
+// vit_create), the lookup is refused while `s` is being captured into a graph, where a symbol
+// lookup (and the module load it may trigger) is not allowed.
+vit_status noalloc_scratch(const vit_model* m, cudaStream_t s, void** ptr) {
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (m->device >= 0 && m->device < 64 && g_noalloc_ptr[m->device] != nullptr) {
+      *ptr = g_noalloc_ptr[m->device];
+      return VIT_OK;
+    }
+  }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  CK(cudaStreamIsCapturing(s, &cs));
+  if (cs != cudaStreamCaptureStatusNone) {
+    set_err("vit_forward_noalloc: the fixed scratch of device %d is not resolved yet and the stream is being "
+            "captured; make one call outside the capture first",
+            m->device);
+    return VIT_E_INVALID_ARG;
+  }
+  const vit_status st = noalloc_resolve(m->device);
+  if (st != VIT_OK) return st;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  *ptr = g_noalloc_ptr[m->device];
   return VIT_OK;
 }
 }  // namespace
@@ -1669,8 +1803,10 @@ extern "C" vit_status vit_forward_noalloc(vit_model* m, const float* images, int
             B, need, kNoAllocScratchBytes);
     return VIT_E_WORKSPACE;
   }
+  st = check_device(m, "vit_forward_noalloc");
+  if (st != VIT_OK) return st;
   void* ws = nullptr;
-  st = noalloc_scratch(&ws);
+  st = noalloc_scratch(m, reinterpret_cast<cudaStream_t>(stream), &ws);
   if (st != VIT_OK) return st;
   const vit_config& c = m->cfg;
   ImgSrc src{images, 3LL * c.img_h * c.img_w, static_cast<long long>(c.img_h) * c.img_w, c.img_w, 1, 0, 0, 0};
