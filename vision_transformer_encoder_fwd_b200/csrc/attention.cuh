@@ -139,10 +139,13 @@ __device__ __forceinline__ void softmax_block_p(const float (&s)[128], float mc,
   }
 }
 
+// kBounded: the launch set a pipeline-wait limit (wait_ns); the default instantiation keeps the
+// fixed 2 s limit out of every wait's fast path.
+template <bool kBounded>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __nv_bfloat16* __restrict__ qkv, int T, int D,
                        __nv_bfloat16* __restrict__ out, int* gstatus, unsigned long long wait_ns) {
-  const unsigned long long wlim = wait_limit(wait_ns);
+  const unsigned long long wlim = kBounded ? wait_ns : 0ull;  // 0: the default limit
   extern __shared__ __align__(1024) uint8_t smem[];
   // The swizzled layouts assume 1024-byte aligned tiles; report and stop if the shared window
   // is not (uniform across the CTA, before anything is allocated).

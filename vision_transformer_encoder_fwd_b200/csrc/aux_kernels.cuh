@@ -21,7 +21,10 @@ struct ImgSrc {
 
 // kornia/dinov3 card "Model I/O" + "DINOv2 n semantic" diagram "Conv2d p x p / p": the
 // patch convolution as a GEMM needs A[b*P + p, k] = bf16(pixel), k = c*p^2 + ky*p + kx, zero
-// for k >= 3 p^2 up to Kpad.  Each thread writes 8 consecutive k (one 16-byte store).
+// for k >= 3 p^2 up to Kpad.  Each thread writes 8 consecutive k (one 16-byte store).  VEC:
+// p is a multiple of 8 and every row start, window origin and stride is a multiple of 4 floats,
+// so the 8 pixels of a thread lie in one image row and load as two 16-byte vectors.
+template <bool VEC>
 __global__ void im2col_bf16_kernel(ImgSrc src, int B, int p, int gw, int P, int Kpad, __nv_bfloat16* __restrict__ A) {
   const int kv = Kpad / 8;
   const long long total = static_cast<long long>(B) * P * kv;
@@ -39,17 +42,34 @@ __global__ void im2col_bf16_kernel(ImgSrc src, int B, int p, int gw, int P, int 
     const int ox = min(ix * src.win_stride, src.max_ox) + gx * p;
     const float* base = src.ptr + b * src.img_stride;
     float v[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int k = k8 * 8 + t;
-      float x = 0.f;
+    if (VEC) {
+      const int k = k8 * 8;
       if (k < K) {
         const int c = k / pp;
         const int rem = k - c * pp;
         const int ky = rem / p, kx = rem - ky * p;
-        x = __ldg(base + c * src.chan_stride + static_cast<long long>(oy + ky) * src.row_stride + (ox + kx));
+        const float4* q = reinterpret_cast<const float4*>(base + c * src.chan_stride +
+                                                          static_cast<long long>(oy + ky) * src.row_stride + (ox + kx));
+        const float4 lo = __ldg(q), hi = __ldg(q + 1);
+        v[0] = lo.x; v[1] = lo.y; v[2] = lo.z; v[3] = lo.w;
+        v[4] = hi.x; v[5] = hi.y; v[6] = hi.z; v[7] = hi.w;
+      } else {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) v[t] = 0.f;
       }
-      v[t] = x;
+    } else {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int k = k8 * 8 + t;
+        float x = 0.f;
+        if (k < K) {
+          const int c = k / pp;
+          const int rem = k - c * pp;
+          const int ky = rem / p, kx = rem - ky * p;
+          x = __ldg(base + c * src.chan_stride + static_cast<long long>(oy + ky) * src.row_stride + (ox + kx));
+        }
+        v[t] = x;
+      }
     }
     uint4 w;
     w.x = pack_bf16x2(v[0], v[1]);

@@ -21,12 +21,6 @@ enum DeviceStatus : int {
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s: far above any real wait
 
-// The pipeline-wait limit a launch asked for (0: the default kWaitTimeoutNs).  Waits that drain
-// copies already in flight on the way out of an aborted kernel always use the default.
-__host__ __device__ __forceinline__ unsigned long long wait_limit(unsigned long long ns) {
-  return ns ? ns : kWaitTimeoutNs;
-}
-
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -55,14 +49,24 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 // One poll of the phase with parity `parity` (the thread may be suspended briefly while the
-// phase is pending).
+// phase is pending).  kHintNs > 0 passes a suspend-time hint: the thread is woken to poll again
+// after at most about that many nanoseconds instead of the system's default.
+template <int kHintNs = 0>
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
+  if (kHintNs > 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "n"(kHintNs)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+  }
   return ok != 0;
 }
 
@@ -81,27 +85,39 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 // (a suspended try_wait could otherwise outlast them).
 constexpr unsigned long long kShortWaitNs = 1000000ull;  // 1 ms
 
+// How a wait polls: kPollDefault suspends in try_wait for the system's default time; kPollSpin
+// spins on the non-blocking test (for a single issuing thread whose reaction time matters more
+// than the issue slots it takes); a positive value is a suspend-time hint in nanoseconds.
+constexpr int kPollDefault = 0;
+constexpr int kPollSpin = -1;
+
 // Wait until the phase of `bar` with parity `parity` has completed.  Gives up (returns false)
-// when the CTA's abort flag is raised by another role or after `limit_ns`; on its own time-out
-// it raises the abort flag and records `site` in the device status word.
+// when the CTA's abort flag is raised by another role or after the wait limit `limit_param`
+// (nanoseconds; 0 selects kWaitTimeoutNs); on its own time-out it raises the abort flag and
+// records `site` in the device status word.  A non-zero limit below kShortWaitNs is polled with
+// the non-blocking test and a clock check on every poll (a suspended try_wait could outlast it).
+template <int kPoll = kPollDefault>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* gstatus, int site, unsigned long long limit_ns = kWaitTimeoutNs) {
-  if (limit_ns < kShortWaitNs) {
+                                          int* gstatus, int site, unsigned long long limit_param = 0) {
+  if (limit_param != 0 && limit_param < kShortWaitNs) {
     const unsigned long long t0 = global_ns();
     for (;;) {
       if (mbar_test_wait(bar, parity)) return true;
       if (*abort_flag) return false;
-      if (global_ns() - t0 > limit_ns) {
+      if (global_ns() - t0 > limit_param) {
         *abort_flag = 1;
         atomicExch(gstatus, site);
         return false;
       }
     }
   }
-  if (mbar_try_wait(bar, parity)) return true;
+  if (kPoll == kPollSpin ? mbar_test_wait(bar, parity) : mbar_try_wait<(kPoll > 0 ? kPoll : 0)>(bar, parity))
+    return true;
+  const unsigned long long limit_ns = limit_param ? limit_param : kWaitTimeoutNs;
   const unsigned long long t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (kPoll == kPollSpin ? mbar_test_wait(bar, parity) : mbar_try_wait<(kPoll > 0 ? kPoll : 0)>(bar, parity))
+      return true;
     if ((it & 31u) == 0) {
       if (*abort_flag) return false;
       if (global_ns() - t0 > limit_ns) {

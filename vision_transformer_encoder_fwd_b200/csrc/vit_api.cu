@@ -269,12 +269,18 @@ cudaError_t launch_gemm(int bn, int mode, const CUtensorMap& a, const CUtensorMa
 
 cudaError_t launch_attention(const CUtensorMap& tm, const __nv_bfloat16* qkv, int B, int T, int heads,
                              __nv_bfloat16* out, int* st, cudaStream_t s, unsigned long long wait_ns) {
-  static std::atomic<uint64_t> attr_done{0};
-  cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel, AttnCfg::SMEM_BYTES, attr_done);
-  if (e != cudaSuccess) return e;
+  static std::atomic<uint64_t> attr_done{0}, attr_done_b{0};
   const int n_qtiles = (T + ATT_BM - 1) / ATT_BM;
   dim3 grid((n_qtiles + ATT_NT - 1) / ATT_NT, heads, B);
-  attn_fwd_tc_kernel<<<grid, ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, qkv, T, heads * 64, out, st, wait_ns);
+  if (wait_ns == 0) {
+    cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel<false>, AttnCfg::SMEM_BYTES, attr_done);
+    if (e != cudaSuccess) return e;
+    attn_fwd_tc_kernel<false><<<grid, ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, qkv, T, heads * 64, out, st, 0ull);
+  } else {
+    cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel<true>, AttnCfg::SMEM_BYTES, attr_done_b);
+    if (e != cudaSuccess) return e;
+    attn_fwd_tc_kernel<true><<<grid, ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, qkv, T, heads * 64, out, st, wait_ns);
+  }
   return cudaGetLastError();
 }
 
@@ -615,8 +621,17 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
 
   // patch embedding: im2col, GEMM with bias + position embedding, token placement
   { const int ps_ = prof_open(m, VIT_K_IM2COL, s);
-  im2col_bf16_kernel<<<grid_1d(static_cast<long long>(Mp) * (m->Kpad / 8), 256, m->nsm), 256, 0, s>>>(
-      src, B, c.patch, g.gw, P, m->Kpad, S.big);
+  {
+    // two 16-byte loads per thread when a thread's 8 pixels are one aligned run of an image row
+    // (K = 3 p^2 is then a multiple of 8 too, so no thread straddles the end of K)
+    const bool vec = c.patch % 8 == 0 && src.img_stride % 4 == 0 && src.chan_stride % 4 == 0 &&
+                     src.row_stride % 4 == 0 && src.win_stride % 4 == 0 && src.max_ox % 4 == 0;
+    const int grid = grid_1d(static_cast<long long>(Mp) * (m->Kpad / 8), 256, m->nsm);
+    if (vec)
+      im2col_bf16_kernel<true><<<grid, 256, 0, s>>>(src, B, c.patch, g.gw, P, m->Kpad, S.big);
+    else
+      im2col_bf16_kernel<false><<<grid, 256, 0, s>>>(src, B, c.patch, g.gw, P, m->Kpad, S.big);
+  }
   prof_close(m, ps_, s); }
   CKL();
   ++launches;
