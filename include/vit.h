@@ -289,7 +289,9 @@ int32_t vit_last_launch_count(const vit_model *m);
  * launch of vit_forward / vit_seg_zero_shot (up to `capacity` launches in total) is bracketed by
  * two CUDA events recorded on the launch stream.  vit_profile_end synchronises those events,
  * adds up the elapsed times per kernel kind into total_ms[VIT_K_COUNT] (milliseconds) and
- * launches[VIT_K_COUNT], and switches profiling off.  Either output pointer may be NULL. */
+ * launches[VIT_K_COUNT], and switches profiling off.  Either output pointer may be NULL.
+ * Launches captured into a CUDA graph while profiling is on keep their events as event-record
+ * nodes: every replay records them again, and vit_profile_end reports the last replay. */
 enum {
   VIT_K_IM2COL = 0, VIT_K_PATCH_GEMM, VIT_K_PREFIX, VIT_K_QKV_GEMM, VIT_K_ATTENTION, VIT_K_PROJ_GEMM,
   VIT_K_FC1_GEMM, VIT_K_FC2_GEMM, VIT_K_TAP, VIT_K_FINAL_LN, VIT_K_SEG_NORM, VIT_K_SEG_COS, VIT_K_SEG_MAP,

@@ -443,11 +443,13 @@ int prof_open(vit_model* m, int kind, cudaStream_t s) {
   if (!m->prof_on || m->prof_used >= static_cast<int>(m->prof_kind.size())) return -1;
   const int slot = m->prof_used++;
   m->prof_kind[slot] = kind;
-  cudaEventRecord(m->prof_ev[2 * slot], s);
+  // external: under stream capture the record becomes an event-record node, which every replay
+  // of the graph records again (outside a capture the flag changes nothing)
+  cudaEventRecordWithFlags(m->prof_ev[2 * slot], s, cudaEventRecordExternal);
   return slot;
 }
 void prof_close(vit_model* m, int slot, cudaStream_t s) {
-  if (slot >= 0) cudaEventRecord(m->prof_ev[2 * slot + 1], s);
+  if (slot >= 0) cudaEventRecordWithFlags(m->prof_ev[2 * slot + 1], s, cudaEventRecordExternal);
   nvtxRangePop();
 }
 
