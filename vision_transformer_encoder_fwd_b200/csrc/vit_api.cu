@@ -438,18 +438,27 @@ const char* const kKindName[VIT_K_COUNT] = {
 // Brackets around one launch: an NVTX range named after the launch kind (seen by Nsight tools
 // when one is attached, a no-op otherwise) and, while per-launch profiling is on and capacity
 // remains, two CUDA events on the launch stream.
+// Under stream capture a profiling record must become an external event-record node, so that
+// every replay of the graph records the event again; outside a capture that flag is refused, and
+// the record is a plain one.
+void prof_record(cudaEvent_t e, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, s);
+}
+
 int prof_open(vit_model* m, int kind, cudaStream_t s) {
   nvtxRangePushA(kKindName[kind]);
   if (!m->prof_on || m->prof_used >= static_cast<int>(m->prof_kind.size())) return -1;
   const int slot = m->prof_used++;
   m->prof_kind[slot] = kind;
-  // external: under stream capture the record becomes an event-record node, which every replay
-  // of the graph records again (outside a capture the flag changes nothing)
-  cudaEventRecordWithFlags(m->prof_ev[2 * slot], s, cudaEventRecordExternal);
+  prof_record(m->prof_ev[2 * slot], s);
   return slot;
 }
 void prof_close(vit_model* m, int slot, cudaStream_t s) {
-  if (slot >= 0) cudaEventRecordWithFlags(m->prof_ev[2 * slot + 1], s, cudaEventRecordExternal);
+  if (slot >= 0) prof_record(m->prof_ev[2 * slot + 1], s);
   nvtxRangePop();
 }
 
