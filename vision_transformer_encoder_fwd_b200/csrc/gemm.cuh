@@ -168,21 +168,33 @@ __device__ __forceinline__ void epi_affine(const EpiParams& ep, float (&v)[32], 
   }
 }
 
-// The row's mean and sum of squared deviations, merged from the producer's partial (mean, M2)
-// pairs in column order; the loads go out eight at a time so their latencies overlap.
+// The row's mean and sum of squared deviations from the producer's partial (mean, M2) pairs.
+// Every partial covers the same nt_cols columns, so the merged mean is the mean of the partial
+// means and M2 = sum_i M2_i + nt_cols * sum_i (mean_i - mean)^2 (the pairwise update of Chan,
+// Golub & LeVeque for equal counts, applied to all partials at once).  The deviations are summed
+// around the first partial's mean, so no division sits in the chain (one reciprocal of nt); the
+// loads go out eight at a time so their latencies overlap.
 __device__ __forceinline__ void merge_row_stats(const EpiParams& ep, int row, float& mu, float& m2out) {
-  float n = 0.f, mean = 0.f, m2 = 0.f;
   const float2* s = ep.stats_in + static_cast<size_t>(row) * ep.nt;
+  float c = 0.f, s1 = 0.f, s2 = 0.f, sm2 = 0.f;
   for (int t0 = 0; t0 < ep.nt; t0 += 8) {
     float2 st[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) st[u] = (t0 + u < ep.nt) ? s[t0 + u] : make_float2(0.f, 0.f);
+    if (t0 == 0) c = st[0].x;
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
-      if (t0 + u < ep.nt) merge_stats(n, mean, m2, static_cast<float>(ep.nt_cols), st[u].x, st[u].y);
+    for (int u = 0; u < 8; ++u) {
+      if (t0 + u < ep.nt) {
+        const float d = st[u].x - c;
+        s1 += d;
+        s2 = fmaf(d, d, s2);
+        sm2 += st[u].y;
+      }
+    }
   }
-  mu = mean;
-  m2out = m2;
+  const float inv = 1.0f / static_cast<float>(ep.nt);
+  mu = c + s1 * inv;
+  m2out = sm2 + static_cast<float>(ep.nt_cols) * fmaxf(fmaf(-s1 * inv, s1, s2), 0.f);
 }
 
 // LNFOLD: rstd of the row and the shift rstd * (ctr - mean) that turns the accumulator of the
