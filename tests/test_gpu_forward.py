@@ -271,3 +271,39 @@ def test_forward_rejects_bad_arguments():
     enc.poll()
     assert torch.equal(desc, before)
     enc.close()
+
+
+_PDL_CHILD = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import synthetic as S, vision_transformer_encoder_fwd_b200 as V
+spec = S.PRESETS["small_s16"]
+enc = V.VitEncoder(spec, S.make_weights(spec, 191), max_batch=2)
+o = enc.forward(S.make_images(spec, 2, 192).cuda(), desc=True, patch=True)
+torch.cuda.synchronize()
+enc.poll()
+np.save(sys.argv[2], o["patch_tokens"].float().cpu().numpy())
+enc.close()
+"""
+
+
+def test_programmatic_dependent_launch_changes_nothing(tmp_path):
+    """The GEMM and attention kernels are launched with programmatic dependent launch unless
+    VIT_B200_PDL=0; a forward in a child process with it off must give the same bits."""
+    need_cuda()
+    import os
+    import subprocess
+    import sys
+    import vision_transformer_encoder_fwd_b200 as V
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = tmp_path / "off.npy"
+    env = dict(os.environ, VIT_B200_PDL="0")
+    subprocess.run([sys.executable, "-c", _PDL_CHILD, root, str(out)], env=env, check=True, timeout=600)
+    spec = S.PRESETS["small_s16"]
+    enc = V.VitEncoder(spec, S.make_weights(spec, 191), max_batch=2)
+    o = enc.forward(S.make_images(spec, 2, 192).cuda(), desc=True, patch=True)
+    torch.cuda.synchronize()
+    enc.poll()
+    on = o["patch_tokens"].float().cpu().numpy()
+    enc.close()
+    assert np.array_equal(on, np.load(out))

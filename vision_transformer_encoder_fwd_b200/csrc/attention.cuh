@@ -176,7 +176,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const int nkv = (T + ATT_BN - 1) / ATT_BN;
 
   if (threadIdx.x == 0) {
-    *abort_flag = (*reinterpret_cast<volatile int*>(gstatus) != 0) ? 1 : 0;
     mbar_init(q_ready, 128 * ntile);
     for (int s = 0; s < ATT_KV_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -206,6 +205,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     tmem_alloc(tmem_holder, AttnCfg::TMEM_COLS);
     tmem_relinquish();
   }
+  // everything above touches only this CTA's shared and tensor memory; global memory from here on
+  pdl_wait();
+  if (threadIdx.x == 0) *abort_flag = (*reinterpret_cast<volatile int*>(gstatus) != 0) ? 1 : 0;
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -21,6 +21,14 @@ enum DeviceStatus : int {
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s: far above any real wait
 
+// Programmatic dependent launch.  pdl_wait: block until the grids this launch depends on have
+// completed and their memory is visible (returns at once when the launch did not allow an early
+// start); nothing before it may touch global memory that an earlier kernel writes or reads.
+// pdl_launch_dependents: let the next kernel of the stream, if launched to allow it, start its
+// own prologue (it is scheduled once every CTA of this grid has started or exited).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

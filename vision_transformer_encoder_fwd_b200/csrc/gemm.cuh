@@ -468,7 +468,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    *abort_flag = (*reinterpret_cast<volatile int*>(gstatus) != 0) ? 1 : 0;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -489,6 +488,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tmem_alloc(tmem_holder, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
+  // everything above touches only this CTA's shared and tensor memory; global memory from here on
+  pdl_wait();
+  if (threadIdx.x == 0) *abort_flag = (*reinterpret_cast<volatile int*>(gstatus) != 0) ? 1 : 0;
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -715,7 +718,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   const bool leader = (rank == 0);
 
   if (threadIdx.x == 0) {
-    *abort_flag = (*reinterpret_cast<volatile int*>(gstatus) != 0) ? 1 : 0;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -736,6 +738,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     tmem_alloc_pair(tmem_holder, Cfg::TMEM_COLS);
     tmem_relinquish_pair();
   }
+  // everything above touches only this cluster's shared and tensor memory; global memory from here on
+  pdl_wait();
+  if (threadIdx.x == 0) *abort_flag = (*reinterpret_cast<volatile int*>(gstatus) != 0) ? 1 : 0;
+  pdl_launch_dependents();
   tc_fence_before();
   cluster_sync_all();
   tc_fence_after();

@@ -17,6 +17,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -181,6 +182,33 @@ cudaError_t set_smem_attr_once(K kernel, int bytes, std::atomic<uint64_t>& done)
   return e;
 }
 
+// Programmatic dependent launch for the tensor-core kernels, which call pdl_wait before they touch
+// global memory: each may be scheduled, and run its prologue (barrier set-up, tensor-memory
+// allocation), while the kernel before it in the stream finishes.  VIT_B200_PDL=0 in the
+// environment launches them in plain stream order instead.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("VIT_B200_PDL");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return on;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, const Args&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int BN, int MODE>
 cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o1, const CUtensorMap& o2,
                           int M, int N, int K, const EpiParams& ep, int* st, cudaStream_t s, int nsm) {
@@ -190,8 +218,8 @@ cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b, const CUte
   if (e != cudaSuccess) return e;
   const int tiles = ((M + GEMM_BM - 1) / GEMM_BM) * (N / BN);
   const int grid = std::max(1, std::min(tiles, nsm));
-  gemm_bf16_tc_kernel<BN, MODE><<<grid, GEMM_THREADS, smem, s>>>(a, b, o1, o2, M, N, K, ep, st);
-  return cudaGetLastError();
+  return launch_pdl(gemm_bf16_tc_kernel<BN, MODE>, dim3(grid), dim3(GEMM_THREADS), smem, s, a, b, o1, o2, M, N, K, ep,
+                    st);
 }
 
 // Tile code for the paired kernel (a 2-CTA cluster per 256 x 256 tile); its B map has 128-row boxes.
@@ -232,8 +260,8 @@ cudaError_t launch_gemm_pair_t(const CUtensorMap& a, const CUtensorMap& b, const
   }
   const int tiles = ((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * ((N + 255) / 256);
   const int clusters = std::max(1, std::min(tiles, mc));
-  gemm_pair_kernel<MODE><<<2 * clusters, GEMM_THREADS, smem, s>>>(a, b, o1, o2, M, N, K, ep, st);
-  return cudaGetLastError();
+  return launch_pdl(gemm_pair_kernel<MODE>, dim3(2 * clusters), dim3(GEMM_THREADS), smem, s, a, b, o1, o2, M, N, K, ep,
+                    st);
 }
 
 // o1 / o2: BIAS, LNFOLD: o1 = bf16 output map (tmap_out_bf16); RESID: o1 = x (tmap_x_f32),
@@ -275,13 +303,14 @@ cudaError_t launch_attention(const CUtensorMap& tm, const __nv_bfloat16* qkv, in
   if (wait_ns == 0) {
     cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel<false>, AttnCfg::SMEM_BYTES, attr_done);
     if (e != cudaSuccess) return e;
-    attn_fwd_tc_kernel<false><<<grid, ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, qkv, T, heads * 64, out, st, 0ull);
+    return launch_pdl(attn_fwd_tc_kernel<false>, grid, dim3(ATT_THREADS), AttnCfg::SMEM_BYTES, s, tm, qkv, T, heads * 64,
+                      out, st, 0ull);
   } else {
     cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel<true>, AttnCfg::SMEM_BYTES, attr_done_b);
     if (e != cudaSuccess) return e;
-    attn_fwd_tc_kernel<true><<<grid, ATT_THREADS, AttnCfg::SMEM_BYTES, s>>>(tm, qkv, T, heads * 64, out, st, wait_ns);
+    return launch_pdl(attn_fwd_tc_kernel<true>, grid, dim3(ATT_THREADS), AttnCfg::SMEM_BYTES, s, tm, qkv, T, heads * 64,
+                      out, st, wait_ns);
   }
-  return cudaGetLastError();
 }
 
 int grid_1d(long long work, int block, int nsm) {
