@@ -26,6 +26,7 @@ struct ImgSrc {
 // so the 8 pixels of a thread lie in one image row and load as two 16-byte vectors.
 template <bool VEC>
 __global__ void im2col_bf16_kernel(ImgSrc src, int B, int p, int gw, int P, int Kpad, __nv_bfloat16* __restrict__ A) {
+  pdl_launch_dependents();
   const int kv = Kpad / 8;
   const long long total = static_cast<long long>(B) * P * kv;
   const int pp = p * p;
@@ -97,6 +98,8 @@ __global__ void token_prep_kernel(const float* __restrict__ cls, const float* __
                                   const float* __restrict__ pos, int pos_on_cls, long long rows, int T, int R, int D,
                                   int gcols, float* __restrict__ x, __nv_bfloat16* __restrict__ xb,
                                   float2* __restrict__ stats, float* __restrict__ ctr) {
+  pdl_wait();  // launched to start early: global memory only after the previous kernel
+  pdl_launch_dependents();
   const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int lane = threadIdx.x & 31;
@@ -222,6 +225,8 @@ __device__ __forceinline__ void row_mean_rstd(const float* __restrict__ xr, int 
 __global__ void final_ln_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ be,
                                 int B, int T, int R, int D, float eps, float* __restrict__ desc, void* __restrict__ patch,
                                 int patch_fp32, int* __restrict__ nonfinite) {
+  pdl_wait();  // launched to start early: global memory only after the previous kernel
+  pdl_launch_dependents();
   const int P = T - 1 - R;
   const int warps_per_block = blockDim.x >> 5;
   const long long job = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5);
@@ -268,6 +273,8 @@ __global__ void final_ln_stream_kernel(float* __restrict__ x, const float* __res
                                        const float* __restrict__ be, long long rows, int D, float eps, int gcols,
                                        __nv_bfloat16* __restrict__ xb, float2* __restrict__ stats,
                                        float* __restrict__ ctr, int* __restrict__ nonfinite) {
+  pdl_wait();  // launched to start early: global memory only after the previous kernel
+  pdl_launch_dependents();
   const int warps_per_block = blockDim.x >> 5;
   const long long row = static_cast<long long>(blockIdx.x) * warps_per_block + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -317,6 +324,8 @@ __global__ void final_ln_stream_kernel(float* __restrict__ x, const float* __res
 // The patch rows of the residual stream, fp32: tok[b, p, :] = x[b, 1 + R + p, :] (the dino.txt
 // head's output tokens, CLS and registers dropped).  float4 copies, grid-stride.
 __global__ void patch_rows_kernel(const float* __restrict__ x, int B, int T, int R, int D, float* __restrict__ tok) {
+  pdl_wait();  // launched to start early: global memory only after the previous kernel
+  pdl_launch_dependents();
   const int P = T - 1 - R;
   const int d4 = D / 4;
   const long long total = static_cast<long long>(B) * P * d4;
@@ -337,6 +346,8 @@ __global__ void patch_rows_kernel(const float* __restrict__ x, int B, int T, int
 // memory so that both the read (along d) and the write (along p) are coalesced.
 __global__ void tap_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ be, int T,
                            int R, int D, float eps, float* __restrict__ out) {
+  pdl_wait();  // launched to start early: global memory only after the previous kernel
+  pdl_launch_dependents();
   __shared__ float tile[32][33];
   __shared__ float s_mean[32], s_rstd[32];
   const int P = T - 1 - R;

@@ -693,8 +693,9 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
     ++launches;
   }
   { const int ps_ = prof_open(m, VIT_K_PREFIX, s);
-  token_prep_kernel<<<(M + 7) / 8, 256, 0, s>>>(m->cls, m->reg, pos, c.pos_on_cls, M, T, R, D, m->stats_cols, S.x,
-                                                 S.xb, S.stats[cur], S.ctr);
+  CK(launch_pdl(token_prep_kernel, dim3(static_cast<unsigned>((M + 7) / 8)), dim3(256), 0, s,
+                static_cast<const float*>(m->cls), static_cast<const float*>(m->reg), pos, c.pos_on_cls,
+                static_cast<long long>(M), T, R, D, m->stats_cols, S.x, S.xb, S.stats[cur], S.ctr));
   prof_close(m, ps_, s); }
   CKL();
   ++launches;
@@ -820,8 +821,9 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
         ++launches;
       } else if (out && out->taps[tap_i]) {
         { const int ps_ = prof_open(m, VIT_K_TAP, s);
-        tap_kernel<<<dim3((P + 31) / 32, B), 256, 0, s>>>(S.x, m->norm_w, m->norm_b, T, R, D, c.ln_eps,
-                                                            out->taps[tap_i]);
+        CK(launch_pdl(tap_kernel, dim3((P + 31) / 32, B), dim3(256), 0, s, static_cast<const float*>(S.x),
+                      static_cast<const float*>(m->norm_w), static_cast<const float*>(m->norm_b), T, R, D, c.ln_eps,
+                      out->taps[tap_i]));
         prof_close(m, ps_, s); }
         CKL();
         ++launches;
@@ -834,9 +836,9 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
     // the head's patch rows (fp32) as the patch tokens
     const long long rows = static_cast<long long>(M);
     { const int ps_ = prof_open(m, VIT_K_FINAL_LN, s);
-    final_ln_stream_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(S.x, m->norm_w, m->norm_b, rows, D, c.ln_eps,
-                                                                          m->stats_cols, S.xb, S.stats[cur], S.ctr,
-                                                                          m->d_status + 1);
+    CK(launch_pdl(final_ln_stream_kernel, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, s, S.x,
+                  static_cast<const float*>(m->norm_w), static_cast<const float*>(m->norm_b), rows, D, c.ln_eps,
+                  m->stats_cols, S.xb, S.stats[cur], S.ctr, m->d_status + 1));
     prof_close(m, ps_, s); }
     CKL();
     ++launches;
@@ -846,8 +848,8 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
     }
     if (out && out->patch_tokens) {
       { const int ps_ = prof_open(m, VIT_K_HEAD_OUT, s);
-      patch_rows_kernel<<<grid_1d(static_cast<long long>(B) * P * (D / 4), 256, m->nsm), 256, 0, s>>>(
-          S.x, B, T, R, D, static_cast<float*>(out->patch_tokens));
+      CK(launch_pdl(patch_rows_kernel, dim3(grid_1d(static_cast<long long>(B) * P * (D / 4), 256, m->nsm)), dim3(256), 0,
+                    s, static_cast<const float*>(S.x), B, T, R, D, static_cast<float*>(out->patch_tokens)));
       prof_close(m, ps_, s); }
       CKL();
       ++launches;
@@ -855,9 +857,10 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
   } else if (out && (out->desc || out->patch_tokens)) {
     const long long jobs = static_cast<long long>(B) * (1 + P);
     { const int ps_ = prof_open(m, VIT_K_FINAL_LN, s);
-    final_ln_kernel<<<static_cast<int>((jobs + 7) / 8), 256, 0, s>>>(S.x, m->norm_w, m->norm_b, B, T, R, D, c.ln_eps,
-                                                                    out->desc, out->patch_tokens, out->patch_fp32,
-                                                                    m->d_status + 1);
+    CK(launch_pdl(final_ln_kernel, dim3(static_cast<unsigned>((jobs + 7) / 8)), dim3(256), 0, s,
+                  static_cast<const float*>(S.x), static_cast<const float*>(m->norm_w),
+                  static_cast<const float*>(m->norm_b), B, T, R, D, c.ln_eps, out->desc, out->patch_tokens,
+                  out->patch_fp32, m->d_status + 1));
     prof_close(m, ps_, s); }
     CKL();
     ++launches;
