@@ -94,3 +94,32 @@ def test_stage_attention_wait_expiry():
             ref = O.attention_probs(q, k) @ v
             err = np.abs(g[bi, :, 64 * h:64 * (h + 1)] - ref).max()
             assert err <= 1e-2 * np.abs(ref).max() + 2e-3, (bi, h, err)
+
+
+def test_stage_attention_wait_expiry_two_tile_ctas():
+    """The same expiry on a grid large enough that each CTA takes two query tiles (ViT-S/14@518
+    batch 8); the next call with the default limit is compared with the oracle on sampled rows."""
+    need_cuda()
+    import vision_transformer_encoder_fwd_b200 as V
+    B, T, heads = 8, 1370, 6
+    D = 64 * heads
+    qkv = S.make_matrix((B, T, 3 * D), 117, 1.0).cuda()
+    out, st = V.stage_attention(qkv, heads, wait_ns=SHORT_NS)
+    torch.cuda.synchronize()
+    code = int(st.item())
+    assert 0x200 < code < 0x300, hex(code)
+    st.zero_()
+    out, st = V.stage_attention(qkv, heads, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    x = qkv.double().cpu().numpy()
+    g = out.double().cpu().numpy()
+    rows = [0, 1, 127, 128, 640, T - 2, T - 1]
+    for bi in (0, B - 1):
+        for h in (0, heads - 1):
+            q = x[bi, rows, 64 * h:64 * (h + 1)]
+            k = x[bi, :, D + 64 * h:D + 64 * (h + 1)]
+            v = x[bi, :, 2 * D + 64 * h:2 * D + 64 * (h + 1)]
+            ref = O.attention_probs(q, k) @ v
+            err = np.abs(g[bi, rows, 64 * h:64 * (h + 1)] - ref).max()
+            assert err <= 6e-3 * np.abs(ref).max() + 1e-3, (bi, h, err)

@@ -5,7 +5,9 @@
 // scaled logits reach ~2.5e6, so Q, K, V and P stay bf16 while the logits, the running maximum
 // and the running sum are fp32 (fp32's exponent range).
 //
-// One CTA per (pair of 128-query tiles, head, image); 10 warps, one CTA per SM:
+// One CTA per (NT 128-query tiles, head, image), NT = 2 (10 warps, one CTA per SM) or NT = 1
+// (6 warps, 256 TMEM columns, two CTAs per SM; faster when the key loop is short, because one
+// CTA's set-up and drain overlap the other's work).  With NT = 2:
 //   warp 0 (one lane)  TMA: K_j and V_j (128 keys x 64 dims each) into a 3-deep ring, read from
 //                      the stacked QKV activation [B, T, 3D] through a 3-D tensor map (rows past
 //                      T are zero-filled).
@@ -27,8 +29,10 @@
 //                      by more than 2^8 (O_i, including its sum column, is then rescaled in TMEM
 //                      first), so every P stays <= 256.
 // TMEM: S_0 [0,128), S_1 [128,256), O_0 [256,336), O_1 [336,416), Q_0 [416,448), Q_1 [448,480)
-// (32-bit columns, lane = row; Q and P hold two bf16 per column).
-// While one softmax group works on S_0 the tensor pipe runs the other tile's MMAs.
+// (32-bit columns, lane = row; Q and P hold two bf16 per column); with NT = 1: S [0,128),
+// O [128,208), Q [208,240) of 256.
+// While one softmax group works on S_0 the tensor pipe runs the other tile's MMAs (NT = 2; with
+// NT = 1 the two CTAs on an SM take that role).
 #pragma once
 
 #include "common.cuh"
@@ -37,8 +41,6 @@ namespace vit {
 
 constexpr int ATT_BM = 128;
 constexpr int ATT_BN = 128;
-constexpr int ATT_NT = 2;  // query tiles per CTA
-constexpr int ATT_THREADS = 320;
 constexpr int ATT_KV_STAGES = 3;
 
 struct AttnCfg {
@@ -51,9 +53,21 @@ struct AttnCfg {
   static constexpr int OFF_BAR = OFF_ONES + V_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 256;
   static_assert(8 * (2 * ATT_KV_STAGES + 10) + 8 <= 256, "barrier area too small");
-  static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int O_COLS = 80;                 // 64 output columns + the sum column + padding
-  static constexpr uint32_t TM_S = 0, TM_O = 256, TM_Q = 416;
+};
+
+// Per-CTA shape for NT query tiles: threads (TMA warp, MMA warp, one softmax warpgroup per
+// tile), TMEM columns and the offsets of the S, O and Q regions.
+template <int NT>
+struct AttnShape {
+  static_assert(NT == 1 || NT == 2, "one or two query tiles per CTA");
+  static constexpr int THREADS = 64 + 128 * NT;
+  static constexpr int MIN_BLOCKS = NT == 1 ? 2 : 1;
+  static constexpr uint32_t TMEM_COLS = NT == 1 ? 256 : 512;
+  static constexpr uint32_t TM_S = 0;
+  static constexpr uint32_t TM_O = 128 * NT;
+  static constexpr uint32_t TM_Q = TM_O + AttnCfg::O_COLS * NT;
+  static_assert(TM_Q + 32 * NT <= TMEM_COLS, "TMEM layout");
 };
 
 // log2(e) / sqrt(64)
@@ -141,8 +155,8 @@ __device__ __forceinline__ void softmax_block_p(const float (&s)[128], float mc,
 
 // kBounded: the launch set a pipeline-wait limit (wait_ns); the default instantiation keeps the
 // fixed 2 s limit out of every wait's fast path.
-template <bool kBounded>
-__global__ void __launch_bounds__(ATT_THREADS, 1)
+template <int NT, bool kBounded>
+__global__ void __launch_bounds__(AttnShape<NT>::THREADS, AttnShape<NT>::MIN_BLOCKS)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __nv_bfloat16* __restrict__ qkv, int T, int D,
                        __nv_bfloat16* __restrict__ out, int* gstatus, unsigned long long wait_ns) {
   const unsigned long long wlim = kBounded ? wait_ns : 0ull;  // 0: the default limit
@@ -169,8 +183,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_qtiles = (T + ATT_BM - 1) / ATT_BM;
-  const int tile0 = blockIdx.x * 2;
-  const int ntile = min(2, n_qtiles - tile0);
+  using Shape = AttnShape<NT>;
+  const int tile0 = blockIdx.x * NT;
+  const int ntile = min(NT, n_qtiles - tile0);
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int nkv = (T + ATT_BN - 1) / ATT_BN;
@@ -202,7 +217,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     fence_proxy_async_smem();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, AttnCfg::TMEM_COLS);
+    tmem_alloc(tmem_holder, Shape::TMEM_COLS);
     tmem_relinquish();
   }
   // everything above touches only this CTA's shared and tensor memory; global memory from here on
@@ -257,11 +272,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
       constexpr uint64_t kStepK = AttnCfg::K_BYTES >> 4;
       constexpr uint64_t kStepV = (AttnCfg::V_BYTES >> 4) - (static_cast<uint64_t>(AttnCfg::V_BYTES >> 4) << 16);
-      const uint32_t t_s0 = tmem_base + AttnCfg::TM_S, t_q0 = tmem_base + AttnCfg::TM_Q;
-      const uint32_t t_o0 = tmem_base + AttnCfg::TM_O;
-      uint32_t aq[2][4], ap[2][8];
+      const uint32_t t_s0 = tmem_base + Shape::TM_S, t_q0 = tmem_base + Shape::TM_Q;
+      const uint32_t t_o0 = tmem_base + Shape::TM_O;
+      uint32_t aq[NT][4], ap[NT][8];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < NT; ++i) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) aq[i][k] = t_q0 + i * 32 + k * 8;
 #pragma unroll
@@ -333,8 +348,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const int q = warp & 3;
       const int r = q * 32 + lane;
       const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-      const uint32_t t_s = tmem_base + lane_off + AttnCfg::TM_S + wg * 128;
-      const uint32_t t_o = tmem_base + lane_off + AttnCfg::TM_O + wg * AttnCfg::O_COLS;
+      const uint32_t t_s = tmem_base + lane_off + Shape::TM_S + wg * 128;
+      const uint32_t t_o = tmem_base + lane_off + Shape::TM_O + wg * AttnCfg::O_COLS;
       {
         // this thread's query row (64 bf16 = 32 columns, two per column) into TMEM
         const int qrow = (tile0 + wg) * ATT_BM + r;
@@ -354,7 +369,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           for (int t = 0; t < 32; ++t) qv[t] = 0u;
         }
         __syncwarp();
-        tmem_st32(tmem_base + lane_off + AttnCfg::TM_Q + wg * 32, qv);
+        tmem_st32(tmem_base + lane_off + Shape::TM_Q + wg * 32, qv);
         tc_fence_before();
         mbar_arrive(q_ready);
       }
@@ -437,7 +452,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (!skip && lane == 0) mbar_wait_drain(mma_done, 0);
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, AttnCfg::TMEM_COLS);
+    tmem_dealloc(tmem_base, Shape::TMEM_COLS);
   }
 }
 
