@@ -190,7 +190,11 @@ __global__ void __launch_bounds__(AttnShape<NT>::THREADS, AttnShape<NT>::MIN_BLO
   const int b = blockIdx.z;
   const int nkv = (T + ATT_BN - 1) / ATT_BN;
 
+  // Launched to start early: wait for the previous kernel before anything else (setting up the
+  // barriers and TMEM first, as the GEMMs do, measured 1.4 % slower here).
+  pdl_wait();
   if (threadIdx.x == 0) {
+    *abort_flag = (*reinterpret_cast<volatile int*>(gstatus) != 0) ? 1 : 0;
     mbar_init(q_ready, 128 * ntile);
     for (int s = 0; s < ATT_KV_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -220,9 +224,6 @@ __global__ void __launch_bounds__(AttnShape<NT>::THREADS, AttnShape<NT>::MIN_BLO
     tmem_alloc(tmem_holder, Shape::TMEM_COLS);
     tmem_relinquish();
   }
-  // everything above touches only this CTA's shared and tensor memory; global memory from here on
-  pdl_wait();
-  if (threadIdx.x == 0) *abort_flag = (*reinterpret_cast<volatile int*>(gstatus) != 0) ? 1 : 0;
   pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
