@@ -26,9 +26,9 @@
  *     head's) also flags any token row holding a NaN or an infinity; vit_poll() then returns
  *     VIT_E_NONFINITE.
  *   - The tensor-core kernels (GEMMs, attention) are launched with programmatic dependent
- *     launch: each may be scheduled and set up its shared and tensor memory while the kernel
- *     before it in the stream finishes, and touches global memory only once that kernel has
- *     completed.  Stream order, graph capture and results are unchanged.  Setting the
+ *     launch: each may be scheduled (the GEMMs also set up their shared and tensor memory)
+ *     while the kernel before it in the stream finishes, and touches global memory only once
+ *     that kernel has completed.  Stream order, graph capture and results are unchanged.  Setting the
  *     environment variable VIT_B200_PDL=0 before the first launch turns it off.
  */
 #ifndef VIT_B200_H
