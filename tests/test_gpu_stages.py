@@ -69,7 +69,7 @@ def _ref_attention(qkv, heads):
     (1, 446, 6, 1.0),     # ViT-S/16@336 tokens
     (2, 1370, 6, 2.0),    # ViT-S/14@518 tokens
     (1, 4101, 2, 1.0),    # ViT-L/16@1024 tokens (two heads)
-    (8, 1370, 6, 1.0),    # ViT-S/14@518 batch 8: enough CTAs that two query tiles share a CTA
+    (8, 1370, 6, 1.0),    # ViT-S/14@518 batch 8: a grid of several waves
 ])
 def test_attention_matches_oracle(B, T, heads, qk_scale):
     need_cuda()

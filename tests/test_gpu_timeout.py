@@ -96,9 +96,9 @@ def test_stage_attention_wait_expiry():
             assert err <= 1e-2 * np.abs(ref).max() + 2e-3, (bi, h, err)
 
 
-def test_stage_attention_wait_expiry_two_tile_ctas():
-    """The same expiry on a grid large enough that each CTA takes two query tiles (ViT-S/14@518
-    batch 8); the next call with the default limit is compared with the oracle on sampled rows."""
+def test_stage_attention_wait_expiry_full_grid():
+    """The same expiry on a grid of several waves (ViT-S/14@518 batch 8, two CTAs per SM); the
+    next call with the default limit is compared with the oracle on sampled rows."""
     need_cuda()
     import vision_transformer_encoder_fwd_b200 as V
     B, T, heads = 8, 1370, 6

@@ -5,42 +5,44 @@
 // scaled logits reach ~2.5e6, so Q, K, V and P stay bf16 while the logits, the running maximum
 // and the running sum are fp32 (fp32's exponent range).
 //
-// One CTA per (NT 128-query tiles, head, image), NT = 2 (10 warps, one CTA per SM) or NT = 1
-// (6 warps, 256 TMEM columns, two CTAs per SM; faster when the key loop is short, because one
-// CTA's set-up and drain overlap the other's work).  With NT = 2:
+// One CTA per (128-query tile, head, image); 6 warps, two CTAs per SM:
 //   warp 0 (one lane)  TMA: K_j and V_j (128 keys x 64 dims each) into a 3-deep ring, read from
 //                      the stacked QKV activation [B, T, 3D] through a 3-D tensor map (rows past
 //                      T are zero-filled).
-//   warp 1             allocates all 512 TMEM columns; one lane issues, per key block j and
-//                      query tile i:  O_i += P_i [V_j | 1]  (A = P_i from TMEM; B = V_j, MN-major,
-//                      extended by a constant column of ones, N = 80), then S_i = Q_i K_{j+1}^T
-//                      with Q_i also read from TMEM, so shared memory only feeds K and V.
-//                      The tensor pipe executes one thread's MMAs in issue order, so S_i may
-//                      overwrite the columns that held P_i.  Column 64 of O_i accumulates
-//                      sum_k P_ik in fp32 -- the softmax denominator of exactly the bf16 P that
-//                      multiplies V.
-//   warps 2..5, 6..9   softmax of query tile 0 and 1, one query row per thread (TMEM lane =
-//                      row).  First each thread copies its Q row from global memory into TMEM.
-//                      Per key block: one 128-column load of S_i, row maximum over the valid
-//                      keys, P = 2^((s - m) log2(e) / 8) -- exponent pairs from one packed fp32
-//                      FMA, the exponential from the special-function unit for most keys and from
-//                      a cubic on the FMA pipe for the rest -- packed to bf16 and written into the
-//                      first 64 columns of S_i.  The running maximum is only moved when it grows
-//                      by more than 2^8 (O_i, including its sum column, is then rescaled in TMEM
-//                      first), so every P stays <= 256.
-// TMEM: S_0 [0,128), S_1 [128,256), O_0 [256,336), O_1 [336,416), Q_0 [416,448), Q_1 [448,480)
-// (32-bit columns, lane = row; Q and P hold two bf16 per column); with NT = 1: S [0,128),
-// O [128,208), Q [208,240) of 256.
-// While one softmax group works on S_0 the tensor pipe runs the other tile's MMAs (NT = 2; with
-// NT = 1 the two CTAs on an SM take that role).
+//   warp 1             allocates 256 TMEM columns; one lane issues the MMAs.  The keys are taken
+//                      in half blocks of 64 (half h of key block j is sub-block 2 j + h), and S has
+//                      two 64-column buffers that the sub-blocks alternate between:
+//                        S_b = Q K_sub^T            (A = Q from TMEM, B = K rows of the half, N = 64)
+//                        O  += P_sub [V_sub | 1]    (A = P from TMEM, B = V rows of the half,
+//                                                    MN-major, extended by a constant column of
+//                                                    ones, N = 80)
+//                      P of a sub-block overwrites the first 32 columns of its own S buffer, and
+//                      the tensor pipe executes one thread's MMAs in issue order, so the S of
+//                      sub-block n + 2 is issued into that buffer right after the PV of
+//                      sub-block n: the S of the next sub-block is always computed while the
+//                      softmax works on the current one.  Column 64 of O accumulates sum_k P_k
+//                      in fp32 -- the softmax denominator of exactly the bf16 P that multiplies V.
+//   warps 2..5         softmax, one query row per thread (TMEM lane = row).  First each thread
+//                      copies its Q row from global memory into TMEM.  Per sub-block: one
+//                      64-column load of S, row maximum over the valid keys, P = 2^((s - m)
+//                      log2(e) / 8) -- exponent pairs from one packed fp32 FMA, the exponential
+//                      from the special-function unit for most keys and from a cubic on the FMA
+//                      pipe for the rest -- packed to bf16 and written over S.  The running
+//                      maximum is only moved when it grows by more than 2^8 (O, including its
+//                      sum column, is then rescaled in TMEM first), so every P stays <= 256.
+// TMEM: S buffers [0,64) and [64,128), O [128,208), Q [208,240) of 256 (32-bit columns, lane =
+// row; Q and P hold two bf16 per column).  Two CTAs share an SM, so one CTA's MMAs run while the
+// other's softmax computes exponentials.
 #pragma once
 
 #include "common.cuh"
 
 namespace vit {
 
-constexpr int ATT_BM = 128;
-constexpr int ATT_BN = 128;
+constexpr int ATT_BM = 128;       // query rows per CTA
+constexpr int ATT_BN = 128;       // keys per TMA stage (two 64-key sub-blocks)
+constexpr int ATT_SUB = 64;       // keys per S buffer
+constexpr int ATT_THREADS = 192;
 constexpr int ATT_KV_STAGES = 3;
 
 struct AttnCfg {
@@ -52,22 +54,12 @@ struct AttnCfg {
   static constexpr int OFF_ONES = OFF_V + ATT_KV_STAGES * V_BYTES;
   static constexpr int OFF_BAR = OFF_ONES + V_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 256;
-  static_assert(8 * (2 * ATT_KV_STAGES + 10) + 8 <= 256, "barrier area too small");
+  static_assert(8 * (2 * ATT_KV_STAGES + 7) + 8 <= 256, "barrier area too small");
+  static constexpr uint32_t TMEM_COLS = 256;
   static constexpr int O_COLS = 80;                 // 64 output columns + the sum column + padding
-};
-
-// Per-CTA shape for NT query tiles: threads (TMA warp, MMA warp, one softmax warpgroup per
-// tile), TMEM columns and the offsets of the S, O and Q regions.
-template <int NT>
-struct AttnShape {
-  static_assert(NT == 1 || NT == 2, "one or two query tiles per CTA");
-  static constexpr int THREADS = 64 + 128 * NT;
-  static constexpr int MIN_BLOCKS = NT == 1 ? 2 : 1;
-  static constexpr uint32_t TMEM_COLS = NT == 1 ? 256 : 512;
-  static constexpr uint32_t TM_S = 0;
-  static constexpr uint32_t TM_O = 128 * NT;
-  static constexpr uint32_t TM_Q = TM_O + AttnCfg::O_COLS * NT;
-  static_assert(TM_Q + 32 * NT <= TMEM_COLS, "TMEM layout");
+  static constexpr uint32_t TM_S = 0, TM_O = 128, TM_Q = 208;
+  // one 64-key sub-block of K or V inside a stage: 64 rows of 128 bytes
+  static constexpr uint64_t kHalfDesc = (ATT_SUB * 128) >> 4;
 };
 
 // log2(e) / sqrt(64)
@@ -101,11 +93,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// Row maximum of 128 logits with four independent 3-input max chains.
-__device__ __forceinline__ float row_max128(const float (&s)[128]) {
+// Row maximum of 64 logits with four independent 3-input max chains.
+__device__ __forceinline__ float row_max64(const float (&s)[64]) {
   float m0 = fmaxf(s[0], s[1]), m1 = fmaxf(s[2], s[3]), m2 = fmaxf(s[4], s[5]), m3 = fmaxf(s[6], s[7]);
 #pragma unroll
-  for (int t = 8; t < 128; t += 8) {
+  for (int t = 8; t < 64; t += 8) {
     m0 = fmax3(m0, s[t], s[t + 1]);
     m1 = fmax3(m1, s[t + 2], s[t + 3]);
     m2 = fmax3(m2, s[t + 4], s[t + 5]);
@@ -114,19 +106,17 @@ __device__ __forceinline__ float row_max128(const float (&s)[128]) {
   return fmax3(m0, m1, fmaxf(m2, m3));
 }
 
-// P for one row of one key block: p = 2^(s * c - m * c) for pairs of keys (one packed fp32 FMA
-// forms the exponent pair); masked keys carry s = -inf and come out as 0 (the FMA-pipe path
-// clamps them to 2^-125 and they are zeroed explicitly).  Each 32-key chunk is packed to bf16
-// and stored to TMEM (16 columns from t_p).  After keys 0..63 the stores are waited for and
-// `half0` is arrived on, so the MMA can start on them while keys 64..127 are computed; `half1`
-// follows the second half.
+// P for one row of a 64-key sub-block: p = 2^(s * c - m * c) for pairs of keys (one packed fp32
+// FMA forms the exponent pair); masked keys carry s = -inf and come out as 0 (the FMA-pipe path
+// clamps them to 2^-125 and they are zeroed explicitly).  The 64 values are packed to bf16 and
+// stored to the first 32 columns of the sub-block's S buffer (t_p); `full` is arrived on once the
+// stores have completed.
 template <bool MASK>
-__device__ __forceinline__ void softmax_block_p(const float (&s)[128], float mc, int valid, uint32_t t_p,
-                                                uint64_t* half0, uint64_t* half1) {
+__device__ __forceinline__ void softmax_sub_p(const float (&s)[64], float mc, int valid, uint32_t t_p, uint64_t* full) {
   const float2 cc = make_float2(kAttnScaleLog2, kAttnScaleLog2);
   const float2 nm = make_float2(-mc, -mc);
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = 0; c < 2; ++c) {
     uint32_t pk[16];
 #pragma unroll
     for (int u = 0; u < 32; u += 2) {
@@ -145,18 +135,16 @@ __device__ __forceinline__ void softmax_block_p(const float (&s)[128], float mc,
       pk[u >> 1] = pack_bf16x2(e.x, e.y);
     }
     tmem_st16_nowait(t_p + c * 16, pk);
-    if (c == 1 || c == 3) {
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(c == 1 ? half0 : half1);
-    }
   }
+  tmem_st_wait();
+  tc_fence_before();
+  mbar_arrive(full);
 }
 
 // kBounded: the launch set a pipeline-wait limit (wait_ns); the default instantiation keeps the
 // fixed 2 s limit out of every wait's fast path.
-template <int NT, bool kBounded>
-__global__ void __launch_bounds__(AttnShape<NT>::THREADS, AttnShape<NT>::MIN_BLOCKS)
+template <bool kBounded>
+__global__ void __launch_bounds__(ATT_THREADS, 2)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __nv_bfloat16* __restrict__ qkv, int T, int D,
                        __nv_bfloat16* __restrict__ out, int* gstatus, unsigned long long wait_ns) {
   const unsigned long long wlim = kBounded ? wait_ns : 0ull;  // 0: the default limit
@@ -172,40 +160,37 @@ __global__ void __launch_bounds__(AttnShape<NT>::THREADS, AttnShape<NT>::MIN_BLO
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnCfg::OFF_BAR);
   uint64_t* kv_full = bars;                               // [ATT_KV_STAGES]
   uint64_t* kv_empty = kv_full + ATT_KV_STAGES;           // [ATT_KV_STAGES]
-  uint64_t* s_full = kv_empty + ATT_KV_STAGES;            // [2]
-  uint64_t* p_full = s_full + 2;                          // [2][2]: tile i, key half h at p_full[2 i + h]
-  uint64_t* pv_done = p_full + 4;                         // [2]
-  uint64_t* mma_done = pv_done + 2;                       // 1
-  uint64_t* q_ready = mma_done + 1;                       // 1: both Q tiles copied into TMEM
+  uint64_t* s_full = kv_empty + ATT_KV_STAGES;            // [2]: S buffer b holds a new sub-block
+  uint64_t* p_full = s_full + 2;                          // [2]: P of the sub-block in buffer b stored
+  uint64_t* pv_done = p_full + 2;                         // 1: the PV MMAs issued so far completed
+  uint64_t* mma_done = pv_done + 1;                       // 1
+  uint64_t* q_ready = mma_done + 1;                       // 1: the Q tile copied into TMEM
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(q_ready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_qtiles = (T + ATT_BM - 1) / ATT_BM;
-  using Shape = AttnShape<NT>;
-  const int tile0 = blockIdx.x * NT;
-  const int ntile = min(NT, n_qtiles - tile0);
+  const int tile = blockIdx.x;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int nkv = (T + ATT_BN - 1) / ATT_BN;
+  const int nsub = (T + ATT_SUB - 1) / ATT_SUB;
 
   // Launched to start early: wait for the previous kernel before anything else (setting up the
-  // barriers and TMEM first, as the GEMMs do, measured 1.4 % slower here).
+  // barriers and TMEM first, as the GEMMs do, measured slower here).
   pdl_wait();
   if (threadIdx.x == 0) {
     *abort_flag = (*reinterpret_cast<volatile int*>(gstatus) != 0) ? 1 : 0;
-    mbar_init(q_ready, 128 * ntile);
+    mbar_init(q_ready, 128);
     for (int s = 0; s < ATT_KV_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[2 * i], 128);
-      mbar_init(&p_full[2 * i + 1], 128);
-      mbar_init(&pv_done[i], 1);
+      mbar_init(&p_full[i], 128);
     }
+    mbar_init(pv_done, 1);
     mbar_init(mma_done, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmQKV);
@@ -221,7 +206,7 @@ __global__ void __launch_bounds__(AttnShape<NT>::THREADS, AttnShape<NT>::MIN_BLO
     fence_proxy_async_smem();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, Shape::TMEM_COLS);
+    tmem_alloc(tmem_holder, AttnCfg::TMEM_COLS);
     tmem_relinquish();
   }
   pdl_launch_dependents();
@@ -233,8 +218,8 @@ __global__ void __launch_bounds__(AttnShape<NT>::THREADS, AttnShape<NT>::MIN_BLO
 
   if (!skip && warp == 0 && lane == 0) {
     // ------------------------------------------------------------------ TMA producer
-    int issued_parity[1 + ATT_KV_STAGES];
-    for (int s = 0; s <= ATT_KV_STAGES; ++s) issued_parity[s] = -1;
+    int issued_parity[ATT_KV_STAGES];
+    for (int s = 0; s < ATT_KV_STAGES; ++s) issued_parity[s] = -1;
     for (int j = 0; j < nkv; ++j) {
       const int s = j % ATT_KV_STAGES;
       const uint32_t ph = static_cast<uint32_t>(j / ATT_KV_STAGES) & 1u;
@@ -242,206 +227,194 @@ __global__ void __launch_bounds__(AttnShape<NT>::THREADS, AttnShape<NT>::MIN_BLO
       mbar_arrive_expect_tx(&kv_full[s], AttnCfg::K_BYTES + AttnCfg::V_BYTES);
       tma_load_3d(sK + s * AttnCfg::K_BYTES, &tmQKV, D + h * 64, j * ATT_BN, b, &kv_full[s]);
       tma_load_3d(sV + s * AttnCfg::V_BYTES, &tmQKV, 2 * D + h * 64, j * ATT_BN, b, &kv_full[s]);
-      issued_parity[1 + s] = static_cast<int>(ph);
+      issued_parity[s] = static_cast<int>(ph);
     }
     if (*abort_flag) {
       for (int s = 0; s < ATT_KV_STAGES; ++s)
-        if (issued_parity[1 + s] >= 0) mbar_wait_drain(&kv_full[s], static_cast<uint32_t>(issued_parity[1 + s]));
+        if (issued_parity[s] >= 0) mbar_wait_drain(&kv_full[s], static_cast<uint32_t>(issued_parity[s]));
     }
   } else if (!skip && warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16(ATT_BM, ATT_BN, false);
+      constexpr uint32_t idesc_s = idesc_bf16(ATT_BM, ATT_SUB, false);
       constexpr uint32_t idesc_o = idesc_bf16(ATT_BM, AttnCfg::O_COLS, true);
       const uint32_t k0 = smem_u32(sK);
       const uint32_t v0 = smem_u32(sV);
       const uint32_t ones0 = smem_u32(smem + AttnCfg::OFF_ONES);
-      // Every MMA operand is built once: K and V descriptors per stage and K step (a K step only
-      // moves the start address: +32 bytes for K, +2048 for V), TMEM addresses per tile.  Each
-      // chain of MMAs into one accumulator is then issued by a single asm statement.
-      // Stage st moves the K start address by st * K_BYTES and the V start address by
-      // st * V_BYTES while the V leading byte offset (distance to the ones atom) shrinks by the
-      // same amount: both are linear in st, so the stage descriptors are one add away.
-      uint64_t dk0[4], dv0[8];
+      // Every MMA operand is built once: K and V descriptors per stage, half and K step (a K step
+      // only moves the start address: +32 bytes for K, +2048 for V), TMEM addresses.  Stage st
+      // moves the K start address by st * K_BYTES and the V start address by st * V_BYTES while
+      // the V leading byte offset (distance to the ones atom) shrinks by the same amount: both are
+      // linear in st, so the stage descriptors are one add away.  The second half of a stage
+      // starts 64 rows (8 KB) later in K, V and the ones atom alike, so only the start moves.
+      uint64_t dk0[4], dv0[4];
       {
         const uint64_t d0 = sdesc_sw128(k0, 16, 1024);
         const uint64_t v0d = sdesc_sw128(v0, ones0 - v0, 1024);
 #pragma unroll
         for (int k = 0; k < 4; ++k) dk0[k] = d0 + 2 * k;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) dv0[kk] = v0d + 128 * kk;
+        for (int kk = 0; kk < 4; ++kk) dv0[kk] = v0d + 128 * kk;
       }
       constexpr uint64_t kStepK = AttnCfg::K_BYTES >> 4;
       constexpr uint64_t kStepV = (AttnCfg::V_BYTES >> 4) - (static_cast<uint64_t>(AttnCfg::V_BYTES >> 4) << 16);
-      const uint32_t t_s0 = tmem_base + Shape::TM_S, t_q0 = tmem_base + Shape::TM_Q;
-      const uint32_t t_o0 = tmem_base + Shape::TM_O;
-      uint32_t aq[NT][4], ap[NT][8];
+      const uint32_t t_s0 = tmem_base + AttnCfg::TM_S, t_q0 = tmem_base + AttnCfg::TM_Q;
+      const uint32_t t_o0 = tmem_base + AttnCfg::TM_O;
+      uint32_t aq[4];
 #pragma unroll
-      for (int i = 0; i < NT; ++i) {
+      for (int k = 0; k < 4; ++k) aq[k] = t_q0 + k * 8;
+      // S of sub-block n (stage (n / 2) % 3, half n % 2) into buffer n % 2
+      auto issue_s = [&](int n) {
+        const int st = (n >> 1) % ATT_KV_STAGES;
+        uint64_t dk[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) aq[i][k] = t_q0 + i * 32 + k * 8;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) ap[i][kk] = t_s0 + i * 128 + kk * 8;
-      }
+        for (int k = 0; k < 4; ++k)
+          dk[k] = dk0[k] + static_cast<uint64_t>(st) * kStepK + ((n & 1) ? AttnCfg::kHalfDesc : 0ull);
+        tc_mma_ts_chain4(t_s0 + ATT_SUB * (n & 1), aq, dk, idesc_s, 0u);
+        tc_commit(&s_full[n & 1]);
+      };
       bool ok = mbar_wait(q_ready, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 2, wlim) &&
                 mbar_wait(&kv_full[0], 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 3, wlim);
       if (ok) {
         tc_fence_after();
-        for (int i = 0; i < ntile; ++i) {
-          tc_mma_ts_chain4(t_s0 + i * 128, aq[i], dk0, idesc_s, 0u);
-          tc_commit(&s_full[i]);
-        }
+        issue_s(0);
+        if (nsub > 1) issue_s(1);
       }
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % ATT_KV_STAGES;
-        const int s1 = (j + 1) % ATT_KV_STAGES;
-        uint64_t dvs[8], dk1[4];
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) dvs[kk] = dv0[kk] + static_cast<uint64_t>(s) * kStepV;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) dk1[k] = dk0[k] + static_cast<uint64_t>(s1) * kStepK;
-        for (int i = 0; i < ntile && ok; ++i) {
-          // P arrives in two halves of 64 keys: the first four PV MMAs run while the softmax
-          // group is still producing the second half.
-          if (!mbar_wait(&p_full[2 * i], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 4, wlim)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          {
-            const uint32_t a_lo[4] = {ap[i][0], ap[i][1], ap[i][2], ap[i][3]};
-            const uint64_t b_lo[4] = {dvs[0], dvs[1], dvs[2], dvs[3]};
-            tc_mma_ts_chain4(t_o0 + i * AttnCfg::O_COLS, a_lo, b_lo, idesc_o, j > 0 ? 1u : 0u);
-          }
-          if (!mbar_wait(&p_full[2 * i + 1], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 9, wlim)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          {
-            const uint32_t a_hi[4] = {ap[i][4], ap[i][5], ap[i][6], ap[i][7]};
-            const uint64_t b_hi[4] = {dvs[4], dvs[5], dvs[6], dvs[7]};
-            tc_mma_ts_chain4(t_o0 + i * AttnCfg::O_COLS, a_hi, b_hi, idesc_o, 1u);
-          }
-          tc_commit(&pv_done[i]);
-          if (j + 1 < nkv) {
-            if (i == 0) {
-              if (!mbar_wait(&kv_full[s1], static_cast<uint32_t>((j + 1) / ATT_KV_STAGES) & 1u, abort_flag, gstatus,
-                             DEV_TIMEOUT_ATTN + 5, wlim)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-            }
-            tc_mma_ts_chain4(t_s0 + i * 128, aq[i], dk1, idesc_s, 0u);
-            tc_commit(&s_full[i]);
-          }
+      for (int n = 0; ok && n < nsub; ++n) {
+        const int buf = n & 1;
+        const int st = (n >> 1) % ATT_KV_STAGES;
+        if (!mbar_wait(&p_full[buf], static_cast<uint32_t>(n >> 1) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 4,
+                       wlim)) {
+          ok = false;
+          break;
         }
-        if (ok) tc_commit(&kv_empty[s]);
+        tc_fence_after();
+        {
+          const uint32_t tp = t_s0 + ATT_SUB * buf;
+          const uint32_t a_p[4] = {tp, tp + 8, tp + 16, tp + 24};
+          uint64_t b_v[4];
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            b_v[kk] = dv0[kk] + static_cast<uint64_t>(st) * kStepV + (buf ? AttnCfg::kHalfDesc : 0ull);
+          tc_mma_ts_chain4(t_o0, a_p, b_v, idesc_o, n > 0 ? 1u : 0u);
+        }
+        tc_commit(pv_done);
+        if (n + 2 < nsub) {
+          // the first half of a new stage: its K and V must have landed
+          if (buf == 0) {
+            const int j2 = (n + 2) >> 1;
+            if (!mbar_wait(&kv_full[j2 % ATT_KV_STAGES], static_cast<uint32_t>(j2 / ATT_KV_STAGES) & 1u, abort_flag,
+                           gstatus, DEV_TIMEOUT_ATTN + 5, wlim)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          issue_s(n + 2);
+        }
+        // both halves of stage st (or the single half of a last, odd stage) are consumed
+        if (buf == 1 || n + 1 == nsub) tc_commit(&kv_empty[st]);
       }
       tc_commit(mma_done);
     }
     __syncwarp();
   } else if (!skip && warp >= 2) {
-    // ------------------------------------------------------------------ softmax groups
-    const int wg = (warp - 2) >> 2;
-    if (wg < ntile) {
-      const int q = warp & 3;
-      const int r = q * 32 + lane;
-      const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-      const uint32_t t_s = tmem_base + lane_off + Shape::TM_S + wg * 128;
-      const uint32_t t_o = tmem_base + lane_off + Shape::TM_O + wg * AttnCfg::O_COLS;
-      {
-        // this thread's query row (64 bf16 = 32 columns, two per column) into TMEM
-        const int qrow = (tile0 + wg) * ATT_BM + r;
-        uint32_t qv[32];
-        if (qrow < T) {
-          const uint4* src = reinterpret_cast<const uint4*>(qkv + (static_cast<size_t>(b) * T + qrow) * (3 * D) + h * 64);
+    // ------------------------------------------------------------------ softmax
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t t_s = tmem_base + lane_off + AttnCfg::TM_S;
+    const uint32_t t_o = tmem_base + lane_off + AttnCfg::TM_O;
+    {
+      // this thread's query row (64 bf16 = 32 columns, two per column) into TMEM
+      const int qrow = tile * ATT_BM + r;
+      uint32_t qv[32];
+      if (qrow < T) {
+        const uint4* src = reinterpret_cast<const uint4*>(qkv + (static_cast<size_t>(b) * T + qrow) * (3 * D) + h * 64);
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const uint4 w = __ldg(src + t);
-            qv[4 * t] = w.x;
-            qv[4 * t + 1] = w.y;
-            qv[4 * t + 2] = w.z;
-            qv[4 * t + 3] = w.w;
-          }
-        } else {
-#pragma unroll
-          for (int t = 0; t < 32; ++t) qv[t] = 0u;
+        for (int t = 0; t < 8; ++t) {
+          const uint4 w = __ldg(src + t);
+          qv[4 * t] = w.x;
+          qv[4 * t + 1] = w.y;
+          qv[4 * t + 2] = w.z;
+          qv[4 * t + 3] = w.w;
         }
-        __syncwarp();
-        tmem_st32(tmem_base + lane_off + Shape::TM_Q + wg * 32, qv);
-        tc_fence_before();
-        mbar_arrive(q_ready);
+      } else {
+#pragma unroll
+        for (int t = 0; t < 32; ++t) qv[t] = 0u;
       }
-      float m = -INFINITY;
-      bool ok = true;
-      for (int j = 0; j < nkv; ++j) {
-        if (!mbar_wait(&s_full[wg], static_cast<uint32_t>(j) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 6, wlim)) {
+      __syncwarp();
+      tmem_st32(tmem_base + lane_off + AttnCfg::TM_Q, qv);
+      tc_fence_before();
+      mbar_arrive(q_ready);
+    }
+    float m = -INFINITY;
+    bool ok = true;
+    for (int n = 0; n < nsub; ++n) {
+      const int buf = n & 1;
+      if (!mbar_wait(&s_full[buf], static_cast<uint32_t>(n >> 1) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 6,
+                     wlim)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[64];
+      __syncwarp();
+      tmem_ld64(t_s + ATT_SUB * buf, s);
+      const int valid = min(ATT_SUB, T - n * ATT_SUB);
+      if (valid < ATT_SUB) {
+#pragma unroll
+        for (int t = 0; t < 64; ++t) s[t] = (t < valid) ? s[t] : -INFINITY;
+      }
+      const float mx = row_max64(s);
+      const float m_new = fmaxf(m, mx);
+      const bool resc = (m_new - m) * kAttnScaleLog2 > kRescaleLog2;
+      float alpha = 1.f;
+      if (resc) {
+        alpha = ex2_approx((m - m_new) * kAttnScaleLog2);
+        m = m_new;
+      }
+      if (n > 0 && __any_sync(0xffffffffu, resc)) {
+        // O holds the sub-blocks before n at the old maximum: wait for the last of them, rescale
+        // (the sum column included) before this sub-block's P is released to the MMA.
+        if (!mbar_wait(pv_done, static_cast<uint32_t>(n - 1) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 7, wlim)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        float s[128];
-        __syncwarp();
-        tmem_ld128(t_s, s);
-        const int valid = min(ATT_BN, T - j * ATT_BN);
-        if (valid < ATT_BN) {
-#pragma unroll
-          for (int t = 0; t < 128; ++t) s[t] = (t < valid) ? s[t] : -INFINITY;
-        }
-        const float mx = row_max128(s);
-        const float m_new = fmaxf(m, mx);
-        const bool resc = (m_new - m) * kAttnScaleLog2 > kRescaleLog2;
-        float alpha = 1.f;
-        if (resc) {
-          alpha = ex2_approx((m - m_new) * kAttnScaleLog2);
-          m = m_new;
-        }
-        if (j > 0 && __any_sync(0xffffffffu, resc)) {
-          // O_i holds the blocks before j at the old maximum: wait for the last of them, rescale
-          // (the sum column included) before any P of block j is released to the MMA.
-          if (!mbar_wait(&pv_done[wg], static_cast<uint32_t>(j - 1) & 1u, abort_flag, gstatus,
-                         DEV_TIMEOUT_ATTN + 7, wlim)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          // 16 columns at a time: the 128 logits stay live in registers meanwhile
 #pragma unroll 1
-          for (int c = 0; c < AttnCfg::O_COLS; c += 16) {
-            float o[16];
-            tmem_ld16(t_o + c, o);
-            uint32_t ob[16];
+        for (int c = 0; c < AttnCfg::O_COLS; c += 16) {
+          float o[16];
+          tmem_ld16(t_o + c, o);
+          uint32_t ob[16];
 #pragma unroll
-            for (int t = 0; t < 16; ++t) ob[t] = __float_as_uint(o[t] * alpha);
-            tmem_st16(t_o + c, ob);
-          }
+          for (int t = 0; t < 16; ++t) ob[t] = __float_as_uint(o[t] * alpha);
+          tmem_st16(t_o + c, ob);
         }
-        const float mc = m * kAttnScaleLog2;
-        __syncwarp();
-        if (valid < ATT_BN)
-          softmax_block_p<true>(s, mc, valid, t_s, &p_full[2 * wg], &p_full[2 * wg + 1]);
-        else
-          softmax_block_p<false>(s, mc, valid, t_s, &p_full[2 * wg], &p_full[2 * wg + 1]);
       }
-      if (ok && mbar_wait(mma_done, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 8, wlim)) {
-        tc_fence_after();
-        float o[64], lsum[16];
-        __syncwarp();
-        tmem_ld64(t_o, o);
-        tmem_ld16(t_o + 64, lsum);
-        const int row = (tile0 + wg) * ATT_BM + r;
-        if (row < T) {
-          const float inv = 1.0f / lsum[0];
-          uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(b) * T + row) * D + h * 64);
+      const float mc = m * kAttnScaleLog2;
+      __syncwarp();
+      if (valid < ATT_SUB)
+        softmax_sub_p<true>(s, mc, valid, t_s + ATT_SUB * buf, &p_full[buf]);
+      else
+        softmax_sub_p<false>(s, mc, valid, t_s + ATT_SUB * buf, &p_full[buf]);
+    }
+    if (ok && mbar_wait(mma_done, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 8, wlim)) {
+      tc_fence_after();
+      float o[64], lsum[16];
+      __syncwarp();
+      tmem_ld64(t_o, o);
+      tmem_ld16(t_o + 64, lsum);
+      const int row = tile * ATT_BM + r;
+      if (row < T) {
+        const float inv = 1.0f / lsum[0];
+        uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(b) * T + row) * D + h * 64);
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            dst[t] = make_uint4(pack_bf16x2(o[8 * t + 0] * inv, o[8 * t + 1] * inv),
-                                pack_bf16x2(o[8 * t + 2] * inv, o[8 * t + 3] * inv),
-                                pack_bf16x2(o[8 * t + 4] * inv, o[8 * t + 5] * inv),
-                                pack_bf16x2(o[8 * t + 6] * inv, o[8 * t + 7] * inv));
-          }
+        for (int t = 0; t < 8; ++t) {
+          dst[t] = make_uint4(pack_bf16x2(o[8 * t + 0] * inv, o[8 * t + 1] * inv),
+                              pack_bf16x2(o[8 * t + 2] * inv, o[8 * t + 3] * inv),
+                              pack_bf16x2(o[8 * t + 4] * inv, o[8 * t + 5] * inv),
+                              pack_bf16x2(o[8 * t + 6] * inv, o[8 * t + 7] * inv));
         }
       }
     }
@@ -453,7 +426,7 @@ __global__ void __launch_bounds__(AttnShape<NT>::THREADS, AttnShape<NT>::MIN_BLO
     if (!skip && lane == 0) mbar_wait_drain(mma_done, 0);
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, Shape::TMEM_COLS);
+    tmem_dealloc(tmem_base, AttnCfg::TMEM_COLS);
   }
 }
 

@@ -295,47 +295,22 @@ cudaError_t launch_gemm(int bn, int mode, const CUtensorMap& a, const CUtensorMa
   }
 }
 
-template <int NT>
-cudaError_t launch_attention_nt(const CUtensorMap& tm, const __nv_bfloat16* qkv, int B, int T, int heads,
-                                __nv_bfloat16* out, int* st, cudaStream_t s, unsigned long long wait_ns) {
+// One CTA per (128-query tile, head, image), two CTAs per SM.
+cudaError_t launch_attention(const CUtensorMap& tm, const __nv_bfloat16* qkv, int B, int T, int heads,
+                             __nv_bfloat16* out, int* st, cudaStream_t s, unsigned long long wait_ns) {
   static std::atomic<uint64_t> attr_done{0}, attr_done_b{0};
-  using Shape = AttnShape<NT>;
   const int n_qtiles = (T + ATT_BM - 1) / ATT_BM;
-  dim3 grid((n_qtiles + NT - 1) / NT, heads, B);
+  dim3 grid(n_qtiles, heads, B);
   if (wait_ns == 0) {
-    cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel<NT, false>, AttnCfg::SMEM_BYTES, attr_done);
+    cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel<false>, AttnCfg::SMEM_BYTES, attr_done);
     if (e != cudaSuccess) return e;
-    return launch_pdl(attn_fwd_tc_kernel<NT, false>, grid, dim3(Shape::THREADS), AttnCfg::SMEM_BYTES, s, tm, qkv, T,
+    return launch_pdl(attn_fwd_tc_kernel<false>, grid, dim3(ATT_THREADS), AttnCfg::SMEM_BYTES, s, tm, qkv, T,
                       heads * 64, out, st, 0ull);
   }
-  cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel<NT, true>, AttnCfg::SMEM_BYTES, attr_done_b);
+  cudaError_t e = set_smem_attr_once(attn_fwd_tc_kernel<true>, AttnCfg::SMEM_BYTES, attr_done_b);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_fwd_tc_kernel<NT, true>, grid, dim3(Shape::THREADS), AttnCfg::SMEM_BYTES, s, tm, qkv, T,
-                    heads * 64, out, st, wait_ns);
-}
-
-// Query tiles per CTA.  Two tiles per CTA (one CTA per SM) is the faster schedule per tile: the
-// MMA issuer serves tile 0 first and tile 1 fills its gaps, which two independent one-tile CTAs
-// on an SM do not do (~10 % more time per tile).  One tile per CTA (two CTAs per SM) wins when it
-// puts fewer tiles on the busiest SM -- few CTAs, or a grid whose last wave of two-tile CTAs is
-// nearly empty -- and, for key loops of at most four blocks, when a later CTA's set-up can
-// overlap an earlier one's work.  Load = tiles on the busiest SM when the CTAs spread evenly.
-int attention_tiles_per_cta(int B, int T, int heads, int nsm) {
-  const long long nq = (T + ATT_BM - 1) / ATT_BM;
-  const int nkv = (T + ATT_BN - 1) / ATT_BN;
-  const long long ctas2 = (nq + 1) / 2 * heads * B;
-  const long long ctas1 = nq * heads * B;
-  const long long load2 = 2 * ((ctas2 + nsm - 1) / nsm);
-  const long long load1 = ctas1 <= nsm ? 1 : 2 * ((ctas1 + 2LL * nsm - 1) / (2LL * nsm));
-  const double per_tile1 = (nkv <= 4 && ctas2 > nsm) ? 0.95 : 1.1;  // relative to a two-tile CTA
-  return static_cast<double>(load1) * per_tile1 < static_cast<double>(load2) ? 1 : 2;
-}
-
-cudaError_t launch_attention(const CUtensorMap& tm, const __nv_bfloat16* qkv, int B, int T, int heads,
-                             __nv_bfloat16* out, int* st, cudaStream_t s, unsigned long long wait_ns, int nsm) {
-  if (attention_tiles_per_cta(B, T, heads, nsm) == 1)
-    return launch_attention_nt<1>(tm, qkv, B, T, heads, out, st, s, wait_ns);
-  return launch_attention_nt<2>(tm, qkv, B, T, heads, out, st, s, wait_ns);
+  return launch_pdl(attn_fwd_tc_kernel<true>, grid, dim3(ATT_THREADS), AttnCfg::SMEM_BYTES, s, tm, qkv, T, heads * 64,
+                    out, st, wait_ns);
 }
 
 int grid_1d(long long work, int block, int nsm) {
@@ -751,7 +726,7 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
       ++launches;
     }
     { const int ps_ = prof_open(m, VIT_K_ATTENTION, s);
-    CK(launch_attention(tm_qkv3, S.big, B, T, c.heads, S.attn, m->d_status, s, m->wait_ns, m->nsm));
+    CK(launch_attention(tm_qkv3, S.big, B, T, c.heads, S.attn, m->d_status, s, m->wait_ns));
     prof_close(m, ps_, s); }
     ++launches;
     // proj + layer scale + residual
@@ -1759,10 +1734,8 @@ vit_status vit_stage_attention_bounded(const void* qkv, int32_t B, int32_t T, in
   }
   CUtensorMap tm;
   if (!tmap_qkv3d(&tm, qkv, B, T, heads * 64)) return VIT_E_CUDA;
-  int dev = 0;
-  CK(cudaGetDevice(&dev));
   CK(launch_attention(tm, static_cast<const __nv_bfloat16*>(qkv), B, T, heads, static_cast<__nv_bfloat16*>(out), status,
-                      reinterpret_cast<cudaStream_t>(stream), wait_ns, device_sms(dev)));
+                      reinterpret_cast<cudaStream_t>(stream), wait_ns));
   return VIT_OK;
 }
 
