@@ -273,13 +273,14 @@ __device__ __forceinline__ void epilogue_store_bf16(const EpiParams& ep, const C
 }
 
 // RESID: one warp's half of a tile.  x arrives by TMA into xbuf[c & 1] (32 rows x 128 bytes, 128B
-// swizzle), chunk c + 1 is requested while chunk c is processed; the updated x goes back into the
+// swizzle), chunk c + 1 is requested while chunk c is processed (XBUF = 1: one buffer, chunk c + 1
+// requested after chunk c is stored, which frees shared memory for a deeper operand ring); the updated x goes back into the
 // same buffer and, with its re-centred bf16 copy bf16(x - centre) (xbbuf: 32 rows x 64 bytes, 64B
 // swizzle), out by TMA stores.  `centre` is this thread's row's mean of x before the update (the
 // same value in every CTA that writes a part of the row); the warps of column group 0 record it
 // in ep.ctr for the folded LayerNorm that reads the copy.  Row statistics (mean, M2) of the new x
 // are written per row for each group of ep.stats_cols columns.
-template <int BN>
+template <int BN, int XBUF = 2>
 __device__ __forceinline__ void epilogue_resid(const EpiParams& ep, const CUtensorMap* tmX, const CUtensorMap* tmXb,
                                                uint32_t taddr, int row0, int n0, float centre, uint8_t* xbuf0,
                                                uint8_t* xbbuf, uint64_t* xfull, uint32_t (&xph)[2],
@@ -293,14 +294,22 @@ __device__ __forceinline__ void epilogue_resid(const EpiParams& ep, const CUtens
   float run_n = 0.f, run_mean = 0.f, run_m2 = 0.f;
 #pragma unroll 1
   for (int c = 0; c < CHUNKS; ++c) {
-    const int buf = c & 1;
+    const int buf = (XBUF == 2) ? (c & 1) : 0;
     const int n = n0 + c * 32;
     if (lane == 0) {
-      tma_store_wait_read0();  // earlier stores have left xbuf[buf ^ 1] and xbbuf
-      if (c + 1 < CHUNKS) {
-        mbar_arrive_expect_tx(&xfull[buf ^ 1], 4096);
-        tma_load_2d(xbuf0 + (buf ^ 1) * 4096, tmX, n + 32, row0, &xfull[buf ^ 1]);
-        xpending[buf ^ 1] = true;
+      tma_store_wait_read0();  // earlier stores have left the x buffer about to be filled and xbbuf
+      if (XBUF == 2) {
+        if (c + 1 < CHUNKS) {
+          mbar_arrive_expect_tx(&xfull[buf ^ 1], 4096);
+          tma_load_2d(xbuf0 + (buf ^ 1) * 4096, tmX, n + 32, row0, &xfull[buf ^ 1]);
+          xpending[buf ^ 1] = true;
+        }
+      } else if (c > 0) {
+        // one buffer: chunk c is requested once chunk c - 1 has been stored (chunk 0 was
+        // requested before the accumulator wait)
+        mbar_arrive_expect_tx(&xfull[0], 4096);
+        tma_load_2d(xbuf0, tmX, n, row0, &xfull[0]);
+        xpending[0] = true;
       }
     }
     __syncwarp();
@@ -658,14 +667,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 //   * each CTA's epilogue reads its own 128 accumulator rows from its own TMEM and releases the
 //     accumulator by arriving (one arrive per warp) on the leader's tempty barrier.
 // No TMA load uses cluster multicast.
-template <int MODE>
+template <int MODE, int XBUF = 2>
 struct PairCfg {
   static constexpr int BN = 256;
-  static constexpr int STAGES = (MODE == EPI_RESID) ? 4 : 6;
+  static constexpr int STAGES = (MODE == EPI_RESID) ? (XBUF == 1 ? 5 : 4) : 6;
   static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
   static constexpr int B_BYTES = (BN / 2) * GEMM_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int EPI_WARP_BYTES = GemmCfg<256, MODE>::EPI_WARP_BYTES;
+  static constexpr int EPI_WARP_BYTES = (MODE == EPI_RESID) ? (XBUF * 4096 + 2048) : GemmCfg<256, MODE>::EPI_WARP_BYTES;
   static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
   static constexpr int OFF_BAR = OFF_EPI + GEMM_EPI_WARPS * EPI_WARP_BYTES;
   static constexpr int BAR_BYTES = 512;
@@ -690,12 +699,12 @@ __device__ __forceinline__ void grace_wait_ns(unsigned long long ns) {
   }
 }
 
-template <int MODE>
+template <int MODE, int XBUF = 2>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmO1, const __grid_constant__ CUtensorMap tmO2, int M, int N,
                      int K, EpiParams ep, int* gstatus) {
-  using Cfg = PairCfg<MODE>;
+  using Cfg = PairCfg<MODE, XBUF>;
   constexpr int BN = Cfg::BN;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -872,8 +881,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                              static_cast<uint32_t>(acc * BN + half * (BN / 2));
       __syncwarp();
       if (MODE == EPI_RESID && active) {
-        epilogue_resid<BN>(ep, &tmO1, &tmO2, taddr, row0, n0, mu, wbuf, wbuf + 8192, wxfull, xph, xpending, abort_flag,
-                           gstatus, ok);
+        epilogue_resid<BN, XBUF>(ep, &tmO1, &tmO2, taddr, row0, n0, mu, wbuf, wbuf + XBUF * 4096, wxfull, xph,
+                                 xpending, abort_flag, gstatus, ok);
         if (!ok) break;
       } else if (MODE != EPI_RESID && active) {
         epilogue_store_bf16<BN, MODE>(ep, &tmO1, taddr, row0, n0, wbuf, mu, rstd);

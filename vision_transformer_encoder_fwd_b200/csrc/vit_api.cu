@@ -224,15 +224,18 @@ cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b, const CUte
 
 // Tile code for the paired kernel (a 2-CTA cluster per 256 x 256 tile); its B map has 128-row boxes.
 constexpr int BN_PAIR = 512;
+// Host-side mode: the residual epilogue with one x buffer per warp and five operand stages
+// (paired tiles; other tilings run EPI_RESID).
+constexpr int EPI_RESID_DEEP = 16;
 
-template <int MODE>
+template <int MODE, int XBUF = 2>
 cudaError_t launch_gemm_pair_t(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o1,
                                const CUtensorMap& o2, int M, int N, int K, const EpiParams& ep, int* st, cudaStream_t s,
                                int nsm) {
   static std::atomic<uint64_t> attr_done{0};
   static std::atomic<int> max_clusters{0};
-  constexpr int smem = PairCfg<MODE>::SMEM_BYTES;
-  cudaError_t e = set_smem_attr_once(gemm_pair_kernel<MODE>, smem, attr_done);
+  constexpr int smem = PairCfg<MODE, XBUF>::SMEM_BYTES;
+  cudaError_t e = set_smem_attr_once(gemm_pair_kernel<MODE, XBUF>, smem, attr_done);
   if (e != cudaSuccess) return e;
   int mc = max_clusters.load();
   if (mc == 0) {
@@ -251,7 +254,7 @@ cudaError_t launch_gemm_pair_t(const CUtensorMap& a, const CUtensorMap& b, const
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<MODE>, &cfg) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<MODE, XBUF>, &cfg) != cudaSuccess || n < 1) {
       cudaGetLastError();
       n = nsm / 2;
     }
@@ -260,7 +263,7 @@ cudaError_t launch_gemm_pair_t(const CUtensorMap& a, const CUtensorMap& b, const
   }
   const int tiles = ((M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * ((N + 255) / 256);
   const int clusters = std::max(1, std::min(tiles, mc));
-  return launch_pdl(gemm_pair_kernel<MODE>, dim3(2 * clusters), dim3(GEMM_THREADS), smem, s, a, b, o1, o2, M, N, K, ep,
+  return launch_pdl(gemm_pair_kernel<MODE, XBUF>, dim3(2 * clusters), dim3(GEMM_THREADS), smem, s, a, b, o1, o2, M, N, K, ep,
                     st);
 }
 
@@ -275,9 +278,11 @@ cudaError_t launch_gemm(int bn, int mode, const CUtensorMap& a, const CUtensorMa
       case EPI_BIAS: return launch_gemm_pair_t<EPI_BIAS>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
       case EPI_LNFOLD: return launch_gemm_pair_t<EPI_LNFOLD>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
       case EPI_RESID: return launch_gemm_pair_t<EPI_RESID>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
+      case EPI_RESID_DEEP: return launch_gemm_pair_t<EPI_RESID, 1>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
       default: return cudaErrorInvalidValue;
     }
   }
+  if (mode == EPI_RESID_DEEP) mode = EPI_RESID;  // the deeper ring is a paired-tile variant only
   if (bn == 256) {
     switch (mode) {
       case EPI_BIAS: return launch_gemm_t<256, EPI_BIAS>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
@@ -794,8 +799,10 @@ vit_status run_forward(vit_model* m, const ImgSrc& src, int B, const Geom& g, co
       ep.stats_cols = m->stats_cols;
       const int bnr = pick_bn_res(M, D, m->bn_res, m->nsm);
       { const int ps_ = prof_open(m, VIT_K_FC2_GEMM, s);
-      CK(launch_gemm(bnr, EPI_RESID, tm_h, bnr == BN_PAIR ? bw.tm_fc2_h : bw.tm_fc2, tm_x_ep, tm_xb_ep, M, D, F, ep,
-                     m->d_status, s, m->nsm));
+      // FC2's long K loop hides its epilogue: one x buffer per warp, the freed shared memory a
+      // fifth operand stage
+      CK(launch_gemm(bnr, EPI_RESID_DEEP, tm_h, bnr == BN_PAIR ? bw.tm_fc2_h : bw.tm_fc2, tm_x_ep, tm_xb_ep, M, D, F,
+                     ep, m->d_status, s, m->nsm));
       prof_close(m, ps_, s); }
       ++launches;
       cur ^= 1;
