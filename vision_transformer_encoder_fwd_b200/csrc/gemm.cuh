@@ -74,7 +74,8 @@ struct EpiParams {
 
 template <int BN, int MODE>
 struct GemmCfg {
-  static constexpr int STAGES = (MODE == EPI_RESID) ? 3 : ((BN == 256) ? 4 : 6);
+  // 128-wide residual tiles have room for a fourth stage (ViT-S/16@336 b64 FC2 71 -> 64 us)
+  static constexpr int STAGES = (MODE == EPI_RESID) ? ((BN == 128) ? 4 : 3) : ((BN == 256) ? 4 : 6);
   static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
   static constexpr int B_BYTES = BN * GEMM_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
