@@ -72,17 +72,19 @@ struct EpiParams {
   int ncls;
 };
 
-template <int BN, int MODE>
+template <int BN, int MODE, int XBUF = 2>
 struct GemmCfg {
-  // 128-wide residual tiles have room for a fourth stage (ViT-S/16@336 b64 FC2 71 -> 64 us)
-  static constexpr int STAGES = (MODE == EPI_RESID) ? ((BN == 128) ? 4 : 3) : ((BN == 256) ? 4 : 6);
+  // 128-wide residual tiles have room for a fourth stage (ViT-S/16@336 b64 FC2 71 -> 64 us), a
+  // fifth with one x buffer per warp (XBUF = 1)
+  static constexpr int STAGES =
+      (MODE == EPI_RESID) ? ((BN == 128) ? (XBUF == 1 ? 5 : 4) : 3) : ((BN == 256) ? 4 : 6);
   static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;
   static constexpr int B_BYTES = BN * GEMM_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   // per epilogue warp: RESID two 32 x 32 fp32 x buffers (128-byte rows, 128B swizzle) and one
   // 32 x 32 bf16 buffer (64-byte rows, 64B swizzle); BIAS / LNFOLD one 32 x 64 bf16 buffer
   static constexpr int EPI_WARP_BYTES =
-      (MODE == EPI_RESID) ? (2 * 4096 + 2048) : ((MODE == EPI_PATCH || MODE == EPI_COS) ? 0 : 4096);
+      (MODE == EPI_RESID) ? (XBUF * 4096 + 2048) : ((MODE == EPI_PATCH || MODE == EPI_COS) ? 0 : 4096);
   static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
   static constexpr int OFF_BAR = OFF_EPI + GEMM_EPI_WARPS * EPI_WARP_BYTES;
   static constexpr int BAR_BYTES = 512;
@@ -453,12 +455,12 @@ __device__ __forceinline__ void epilogue_cos(const EpiParams& ep, uint32_t taddr
 // tmO1 / tmO2: BIAS / LNFOLD -> tmO1 = output [M, ldo] bf16 (box 64 x 32, 128B swizzle);
 //              RESID -> tmO1 = x [M, N] fp32 (box 32 x 32, 128B swizzle), tmO2 = xb [M, N] bf16
 //              (box 32 x 32, 64B swizzle); PATCH -> unused.
-template <int BN, int MODE>
+template <int BN, int MODE, int XBUF = 2>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmO1, const __grid_constant__ CUtensorMap tmO2, int M,
                         int N, int K, EpiParams ep, int* gstatus) {
-  using Cfg = GemmCfg<BN, MODE>;
+  using Cfg = GemmCfg<BN, MODE, XBUF>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -617,7 +619,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                              static_cast<uint32_t>(acc * BN + half * (BN / 2));
       __syncwarp();
       if (MODE == EPI_RESID) {
-        epilogue_resid<BN>(ep, &tmO1, &tmO2, taddr, row0, n0, mu, wbuf, wbuf + 8192, wxfull, xph, xpending, abort_flag,
+        epilogue_resid<BN, XBUF>(ep, &tmO1, &tmO2, taddr, row0, n0, mu, wbuf, wbuf + XBUF * 4096, wxfull, xph, xpending, abort_flag,
                            gstatus, ok);
         if (!ok) break;
       } else if (MODE == EPI_PATCH) {

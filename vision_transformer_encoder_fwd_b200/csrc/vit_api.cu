@@ -209,23 +209,23 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <int BN, int MODE>
+template <int BN, int MODE, int XBUF = 2>
 cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o1, const CUtensorMap& o2,
                           int M, int N, int K, const EpiParams& ep, int* st, cudaStream_t s, int nsm) {
   static std::atomic<uint64_t> attr_done{0};
-  constexpr int smem = GemmCfg<BN, MODE>::SMEM_BYTES;
-  cudaError_t e = set_smem_attr_once(gemm_bf16_tc_kernel<BN, MODE>, smem, attr_done);
+  constexpr int smem = GemmCfg<BN, MODE, XBUF>::SMEM_BYTES;
+  cudaError_t e = set_smem_attr_once(gemm_bf16_tc_kernel<BN, MODE, XBUF>, smem, attr_done);
   if (e != cudaSuccess) return e;
   const int tiles = ((M + GEMM_BM - 1) / GEMM_BM) * (N / BN);
   const int grid = std::max(1, std::min(tiles, nsm));
-  return launch_pdl(gemm_bf16_tc_kernel<BN, MODE>, dim3(grid), dim3(GEMM_THREADS), smem, s, a, b, o1, o2, M, N, K, ep,
-                    st);
+  return launch_pdl(gemm_bf16_tc_kernel<BN, MODE, XBUF>, dim3(grid), dim3(GEMM_THREADS), smem, s, a, b, o1, o2, M, N, K,
+                    ep, st);
 }
 
 // Tile code for the paired kernel (a 2-CTA cluster per 256 x 256 tile); its B map has 128-row boxes.
 constexpr int BN_PAIR = 512;
-// Host-side mode: the residual epilogue with one x buffer per warp and five operand stages
-// (paired tiles; other tilings run EPI_RESID).
+// Host-side mode: the residual epilogue with one x buffer per warp and one more operand stage
+// (paired and 128-wide tiles; 128 x 256 tiles run EPI_RESID).
 constexpr int EPI_RESID_DEEP = 16;
 
 template <int MODE, int XBUF = 2>
@@ -282,7 +282,9 @@ cudaError_t launch_gemm(int bn, int mode, const CUtensorMap& a, const CUtensorMa
       default: return cudaErrorInvalidValue;
     }
   }
-  if (mode == EPI_RESID_DEEP) mode = EPI_RESID;  // the deeper ring is a paired-tile variant only
+  if (mode == EPI_RESID_DEEP && bn == 128)
+    return launch_gemm_t<128, EPI_RESID, 1>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
+  if (mode == EPI_RESID_DEEP) mode = EPI_RESID;  // 128 x 256 tiles have no room for a deeper ring
   if (bn == 256) {
     switch (mode) {
       case EPI_BIAS: return launch_gemm_t<256, EPI_BIAS>(a, b, o1, o2, M, N, K, ep, st, s, nsm);
