@@ -6,14 +6,14 @@
 // and the running sum are fp32 (fp32's exponent range).
 //
 // One CTA per (128-query tile, head, image); 6 warps, two CTAs per SM:
-//   warp 0 (one lane)  TMA: K_j and V_j (128 keys x 64 dims each) into a 3-deep ring, read from
+//   warp 0 (one lane)  TMA: K_n and V_n (64 keys x 64 dims each) into a 6-deep ring, read from
 //                      the stacked QKV activation [B, T, 3D] through a 3-D tensor map (rows past
 //                      T are zero-filled).
 //   warp 1             allocates 256 TMEM columns; one lane issues the MMAs.  The keys are taken
-//                      in half blocks of 64 (half h of key block j is sub-block 2 j + h), and S has
-//                      two 64-column buffers that the sub-blocks alternate between:
-//                        S_b = Q K_sub^T            (A = Q from TMEM, B = K rows of the half, N = 64)
-//                        O  += P_sub [V_sub | 1]    (A = P from TMEM, B = V rows of the half,
+//                      in sub-blocks of 64, and S has two 64-column buffers that the sub-blocks
+//                      alternate between:
+//                        S_b = Q K_n^T              (A = Q from TMEM, B = K_n, N = 64)
+//                        O  += P_n [V_n | 1]        (A = P from TMEM, B = V_n,
 //                                                    MN-major, extended by a constant column of
 //                                                    ones, N = 80)
 //                      P of a sub-block overwrites the first 32 columns of its own S buffer, and
@@ -40,14 +40,14 @@
 namespace vit {
 
 constexpr int ATT_BM = 128;       // query rows per CTA
-constexpr int ATT_BN = 128;       // keys per TMA stage (two 64-key sub-blocks)
+constexpr int ATT_BN = 64;        // keys per TMA stage: one sub-block
 constexpr int ATT_SUB = 64;       // keys per S buffer
 constexpr int ATT_THREADS = 192;
-constexpr int ATT_KV_STAGES = 3;
+constexpr int ATT_KV_STAGES = 6;  // (three 128-key stages measured 3.5 % slower at ViT-L/16@1024 b8)
 
 struct AttnCfg {
-  static constexpr int K_BYTES = ATT_BN * 64 * 2;   // 16 KB
-  static constexpr int V_BYTES = ATT_BN * 64 * 2;   // 16 KB
+  static constexpr int K_BYTES = ATT_BN * 64 * 2;   // 8 KB
+  static constexpr int V_BYTES = ATT_BN * 64 * 2;   // 8 KB
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + ATT_KV_STAGES * K_BYTES;
   // the constant "ones" MN-major atom that extends every V stage by 16 columns (1, 0, ..., 0)
@@ -58,8 +58,6 @@ struct AttnCfg {
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr int O_COLS = 80;                 // 64 output columns + the sum column + padding
   static constexpr uint32_t TM_S = 0, TM_O = 128, TM_Q = 208;
-  // one 64-key sub-block of K or V inside a stage: 64 rows of 128 bytes
-  static constexpr uint64_t kHalfDesc = (ATT_SUB * 128) >> 4;
 };
 
 // log2(e) / sqrt(64)
@@ -198,7 +196,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     tma_prefetch_desc(&tmQKV);
   }
   {
-    // The ones atom: 128 key rows of 128 bytes in the 128-byte-swizzled MN-major layout, value
+    // The ones atom: 64 key rows of 128 bytes in the 128-byte-swizzled MN-major layout, value
     // 1.0 at N position 0 of every row (16-byte chunk 0, swizzled to chunk r % 8), 0 elsewhere.
     uint4* ones = reinterpret_cast<uint4*>(smem + AttnCfg::OFF_ONES);
     for (int i = threadIdx.x; i < AttnCfg::V_BYTES / 16; i += blockDim.x) {
@@ -243,12 +241,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       const uint32_t k0 = smem_u32(sK);
       const uint32_t v0 = smem_u32(sV);
       const uint32_t ones0 = smem_u32(smem + AttnCfg::OFF_ONES);
-      // Every MMA operand is built once: K and V descriptors per stage, half and K step (a K step
-      // only moves the start address: +32 bytes for K, +2048 for V), TMEM addresses.  Stage st
-      // moves the K start address by st * K_BYTES and the V start address by st * V_BYTES while
-      // the V leading byte offset (distance to the ones atom) shrinks by the same amount: both are
-      // linear in st, so the stage descriptors are one add away.  The second half of a stage
-      // starts 64 rows (8 KB) later in K, V and the ones atom alike, so only the start moves.
+      // Every MMA operand is built once: K and V descriptors per stage and K step (a K step only
+      // moves the start address: +32 bytes for K, +2048 for V), TMEM addresses.  Stage st moves
+      // the K start address by st * K_BYTES and the V start address by st * V_BYTES while the V
+      // leading byte offset (distance to the ones atom) shrinks by the same amount: both are
+      // linear in st, so the stage descriptors are one add away.
       uint64_t dk0[4], dv0[4];
       {
         const uint64_t d0 = sdesc_sw128(k0, 16, 1024);
@@ -265,13 +262,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       uint32_t aq[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) aq[k] = t_q0 + k * 8;
-      // S of sub-block n (stage (n / 2) % 3, half n % 2) into buffer n % 2
+      // S of sub-block n (stage n % ATT_KV_STAGES) into buffer n % 2
       auto issue_s = [&](int n) {
-        const int st = (n >> 1) % ATT_KV_STAGES;
+        const int st = n % ATT_KV_STAGES;
         uint64_t dk[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          dk[k] = dk0[k] + static_cast<uint64_t>(st) * kStepK + ((n & 1) ? AttnCfg::kHalfDesc : 0ull);
+        for (int k = 0; k < 4; ++k) dk[k] = dk0[k] + static_cast<uint64_t>(st) * kStepK;
         tc_mma_ts_chain4(t_s0 + ATT_SUB * (n & 1), aq, dk, idesc_s, 0u);
         tc_commit(&s_full[n & 1]);
       };
@@ -280,11 +276,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       if (ok) {
         tc_fence_after();
         issue_s(0);
-        if (nsub > 1) issue_s(1);
+      }
+      if (ok && nsub > 1) {
+        ok = mbar_wait(&kv_full[1], 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 3, wlim);
+        if (ok) {
+          tc_fence_after();
+          issue_s(1);
+        }
       }
       for (int n = 0; ok && n < nsub; ++n) {
         const int buf = n & 1;
-        const int st = (n >> 1) % ATT_KV_STAGES;
+        const int st = n % ATT_KV_STAGES;
         if (!mbar_wait(&p_full[buf], static_cast<uint32_t>(n >> 1) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 4,
                        wlim)) {
           ok = false;
@@ -297,25 +299,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
           uint64_t b_v[4];
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            b_v[kk] = dv0[kk] + static_cast<uint64_t>(st) * kStepV + (buf ? AttnCfg::kHalfDesc : 0ull);
+            b_v[kk] = dv0[kk] + static_cast<uint64_t>(st) * kStepV;
           tc_mma_ts_chain4(t_o0, a_p, b_v, idesc_o, n > 0 ? 1u : 0u);
         }
         tc_commit(pv_done);
         if (n + 2 < nsub) {
-          // the first half of a new stage: its K and V must have landed
-          if (buf == 0) {
-            const int j2 = (n + 2) >> 1;
-            if (!mbar_wait(&kv_full[j2 % ATT_KV_STAGES], static_cast<uint32_t>(j2 / ATT_KV_STAGES) & 1u, abort_flag,
-                           gstatus, DEV_TIMEOUT_ATTN + 5, wlim)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
+          const int j2 = n + 2;
+          if (!mbar_wait(&kv_full[j2 % ATT_KV_STAGES], static_cast<uint32_t>(j2 / ATT_KV_STAGES) & 1u, abort_flag,
+                         gstatus, DEV_TIMEOUT_ATTN + 5, wlim)) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
           issue_s(n + 2);
         }
-        // both halves of stage st (or the single half of a last, odd stage) are consumed
-        if (buf == 1 || n + 1 == nsub) tc_commit(&kv_empty[st]);
+        tc_commit(&kv_empty[st]);
       }
       tc_commit(mma_done);
     }
