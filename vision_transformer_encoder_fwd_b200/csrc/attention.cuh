@@ -235,6 +235,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     }
   } else if (!skip && warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
+    // (its waits poll with a 32 ns suspend-time hint: 0-4 % faster than the default suspension on
+    // the measured shapes, the softmax and TMA waits keep the default)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(ATT_BM, ATT_SUB, false);
       constexpr uint32_t idesc_o = idesc_bf16(ATT_BM, AttnCfg::O_COLS, true);
@@ -271,14 +273,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
         tc_mma_ts_chain4(t_s0 + ATT_SUB * (n & 1), aq, dk, idesc_s, 0u);
         tc_commit(&s_full[n & 1]);
       };
-      bool ok = mbar_wait(q_ready, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 2, wlim) &&
-                mbar_wait(&kv_full[0], 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 3, wlim);
+      bool ok = mbar_wait<32>(q_ready, 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 2, wlim) &&
+                mbar_wait<32>(&kv_full[0], 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 3, wlim);
       if (ok) {
         tc_fence_after();
         issue_s(0);
       }
       if (ok && nsub > 1) {
-        ok = mbar_wait(&kv_full[1], 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 3, wlim);
+        ok = mbar_wait<32>(&kv_full[1], 0, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 3, wlim);
         if (ok) {
           tc_fence_after();
           issue_s(1);
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       for (int n = 0; ok && n < nsub; ++n) {
         const int buf = n & 1;
         const int st = n % ATT_KV_STAGES;
-        if (!mbar_wait(&p_full[buf], static_cast<uint32_t>(n >> 1) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 4,
+        if (!mbar_wait<32>(&p_full[buf], static_cast<uint32_t>(n >> 1) & 1u, abort_flag, gstatus, DEV_TIMEOUT_ATTN + 4,
                        wlim)) {
           ok = false;
           break;
@@ -305,7 +307,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
         tc_commit(pv_done);
         if (n + 2 < nsub) {
           const int j2 = n + 2;
-          if (!mbar_wait(&kv_full[j2 % ATT_KV_STAGES], static_cast<uint32_t>(j2 / ATT_KV_STAGES) & 1u, abort_flag,
+          if (!mbar_wait<32>(&kv_full[j2 % ATT_KV_STAGES], static_cast<uint32_t>(j2 / ATT_KV_STAGES) & 1u, abort_flag,
                          gstatus, DEV_TIMEOUT_ATTN + 5, wlim)) {
             ok = false;
             break;
