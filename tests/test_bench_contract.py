@@ -80,3 +80,47 @@ def _timed(fn):
     t0 = time.perf_counter()
     fn()
     return time.perf_counter() - t0
+
+
+def test_clock_sampler_summarises_only_the_timed_window(monkeypatch):
+    """The sampler waits for nvidia-smi's first line, and mark() opens the window that stop()
+    summarises: samples taken before the timed region (an idle clock) are left out, throttle
+    reasons inside it are reported."""
+    import io
+    import time as _time
+    pre = "0, 1965, 1965, 120.5, 0x0, Not Active, Not Active, Not Active, Not Active\n"
+    inside = ["0, 1700, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, Active\n",
+              "0, 1680, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active\n",
+              "0, 1720, 1965, 940.0, 0x4, Not Active, Not Active, Not Active, Active\n"]
+
+    class FakeProc:
+        def __init__(self, *a, **k):
+            self.stdout = io.StringIO(pre)
+            self.alive = True
+
+        def poll(self):
+            return None if self.alive else 0
+
+        def terminate(self):
+            self.alive = False
+
+        def wait(self, timeout=None):
+            return 0
+
+        def kill(self):
+            self.alive = False
+
+    monkeypatch.setattr(bench.subprocess, "Popen", FakeProc)
+    cs = bench.ClockSampler(0)
+    cs.start()
+    t0 = _time.time()
+    while not cs.lines and _time.time() - t0 < 2:
+        _time.sleep(0.01)
+    assert cs.lines == [pre.strip()]
+    cs.mark()
+    cs.lines.extend(x.strip() for x in inside)     # what the reader thread appends meanwhile
+    clk = cs.stop()
+    assert clk["samples"] == 3
+    assert clk["sm_mhz"] == 1700.0 and clk["sm_max_mhz"] == 1965.0
+    assert clk["reasons"] == ["sw_power_cap"]
+    assert clk["power_w"] == 940.0
